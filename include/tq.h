@@ -1,0 +1,246 @@
+/*
+ * tq.h — C ABI of the B200 compressed-KV library (libtq.so).
+ *
+ * The library computes the TurboQuant / TurboESM key-value cache path:
+ *   RoPE -> orthogonal rotation Pi -> per-vector fp32 norm + b-bit Lloyd-Max
+ *   index per coordinate -> (keys) 1-bit QJL sign sketch of the residual plus
+ *   the residual norm -> attention computed directly over the packed cache.
+ * Sources: gist.science "TurboESM: Ultra-Efficient 3-Bit KV Cache Quantization
+ * for Protein Language Models with Orthogonal Rotation and QJL Correction"
+ * (technical summary, sections 2A-2E) and 7minutos.es "KV cache está
+ * consumiendo tu VRAM ... TurboQuant" (Etapa 1 and Etapa 2).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers documented "device" must point to memory of the current CUDA
+ *    device; "host" pointers to ordinary host memory. The caller owns every
+ *    buffer; the library allocates nothing.
+ *  - Every GPU call is asynchronous on the given stream (`stream` is a
+ *    cudaStream_t passed as void*; NULL = legacy default stream).
+ *  - Arguments are validated on the host; on any violation the call returns
+ *    TQ_ERR_INVALID_ARG (or TQ_ERR_UNSUPPORTED) without launching anything.
+ *    tq_last_error_string() then describes the problem (per host thread).
+ *  - Kernels never trap. Conditions only the device can see are OR-ed into
+ *    the optional device word *d_status (TQ_DEV_* bits); read it after the
+ *    stream has synchronised. A NULL d_status disables that reporting.
+ *  - Pi and S are data (seeded by the caller); the library draws no random
+ *    numbers.
+ *
+ * Packed-cache layout (one "row" per vector, rows of a plane are contiguous)
+ * -------------------------------------------------------------------------
+ *  index plane  uint8  [n][d*bits/8]   8 coordinates per `bits` bytes; the
+ *               group of coordinates 8g..8g+7, read as a little-endian integer,
+ *               holds code[8g+j] at bits [bits*j, bits*j+bits).
+ *  sign plane   uint32 [n][ceil(d/32)] (keys) bit i of the sketch at bit
+ *               (i mod 32) of word i/32; pad bits are 0.
+ *  norm plane   float  [n]             ||x|| of the (RoPE'd) input vector.
+ *  rnorm plane  float  [n]             (keys) ||r||, r = Pi x - ||x|| c[code].
+ * A cache for [B][H][N] vectors stores row (b*H + h)*ctx_stride + t.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or combination   */
+  TQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement   */
+  TQ_ERR_CUDA = 3,          /* a CUDA runtime call failed (see error string)  */
+  TQ_ERR_WORKSPACE = 4      /* workspace missing or smaller than required    */
+} tq_status;
+
+/* Device-side status bits OR-ed into *d_status. */
+#define TQ_DEV_BAD_CODEBOOK   0x1  /* boundaries not strictly increasing       */
+#define TQ_DEV_BAD_POSITION   0x2  /* a RoPE position was negative            */
+#define TQ_DEV_TIMEOUT        0x4  /* a kernel gave up waiting on its own pipeline
+                                      (bounded wait); outputs of that call are invalid */
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/* Shape of one head's packed vectors. d: head dim, a multiple of 8 in
+ * [8, 256]; key_bits / value_bits: index bits per coordinate, 2..4. */
+typedef struct {
+  int32_t d;
+  int32_t key_bits;
+  int32_t value_bits;
+} tq_layout;
+
+/* The planes of one packed tensor (all device pointers; 16-byte aligned).
+ * sign and rnorm are used for keys only and may be NULL for values. */
+typedef struct {
+  uint8_t*  idx;
+  uint32_t* sign;
+  float*    norm;
+  float*    rnorm;
+} tq_planes;
+
+/* ------------------------------------------------------------------------
+ * Sizes of the packed layout.
+ * ---------------------------------------------------------------------- */
+/* Bytes of one index row: d*bits/8. */
+int64_t tq_idx_row_bytes(int32_t d, int32_t bits);
+/* 32-bit words of one sign row: ceil(d/32). */
+int64_t tq_sign_words(int32_t d);
+/* Total packed bytes of n vectors (index + sign + norm + rnorm planes for a
+ * key, index + norm planes for a value). -1 on invalid arguments. */
+int64_t tq_packed_bytes(const tq_layout* layout, int64_t n_vectors, int32_t is_key);
+
+/* ------------------------------------------------------------------------
+ * tq_make_codebook — Lloyd-Max levels for one coordinate (host only).
+ *
+ * 7minutos.es "KV cache ... TurboQuant", Etapa 1: after a random rotation a
+ * coordinate x of a unit vector follows x^2 ~ Beta(1/2, (d-1)/2), density
+ * proportional to (1-x^2)^((d-3)/2) on [-1,1]; Lloyd-Max alternates
+ * "boundary = midpoint of adjacent levels" and "level = mean of its cell"
+ * until the error stops improving; the codebook depends only on (d, bits).
+ * gist.science TurboESM section 2C: K and V get separate tables fitted to
+ * their own post-rotation coordinates ("dual LUT") — mode 1.
+ *
+ *  d            >= 3 (mode 0); ignored for mode 1
+ *  bits         1..4 (2^bits levels)
+ *  mode         0 = analytic law above; 1 = empirical Lloyd on `samples`
+ *  samples      host, n_samples floats (mode 1 only; coordinates of rotated
+ *               unit vectors); NULL for mode 0
+ *  centroids    host out, 2^bits floats, strictly increasing
+ *  boundaries   host out, 2^bits - 1 floats, midpoints of adjacent centroids
+ *               (computed in double, then rounded)
+ *  mse_out      host out (nullable): per-coordinate distortion (mode 0: under
+ *               the law; mode 1: over the samples)
+ * Start: the 2^bits equiprobable quantiles. Stop: no level moves by 1e-13
+ * (mode 0; the result is then made exactly symmetric) or no sample changes
+ * cell (mode 1). Errors: TQ_ERR_INVALID_ARG.
+ * ---------------------------------------------------------------------- */
+tq_status tq_make_codebook(int32_t d, int32_t bits, int32_t mode,
+                           const float* samples, int64_t n_samples,
+                           float* centroids, float* boundaries, double* mse_out);
+
+/* ------------------------------------------------------------------------
+ * tq_quantize_kv — quantise and pack n vectors (one launch; device).
+ *
+ * gist.science TurboESM section 2A: RoPE first, then the orthogonal Pi.
+ * 7minutos.es Etapa 1: y = Pi x, each coordinate of y/||x|| replaced by the
+ * index of its Lloyd-Max level. Etapa 2 (keys): the residual of stage 1 is
+ * multiplied by the Gaussian S; the signs of the result (1 bit each) and the
+ * residual's L2 norm are stored.
+ *
+ * Per vector v (row v of x):
+ *   x'   = RoPE(x_v, positions[v])   rotate-half pairs (i, i+d/2) turned by
+ *                                    positions[v] * rope_base^(-2i/d);
+ *                                    skipped when positions==NULL or
+ *                                    rope_base <= 0
+ *   y    = Pi_g x'                   g = v / vectors_per_pi
+ *   code_i = #{ j : y_i > ||x'|| * boundaries[j] }   (ties go to the lower code)
+ *   keys: r = y - ||x'|| centroids[code];  sign_i = ((S r)_i >= 0)
+ * Codes and signs equal those of exact arithmetic: any coordinate (or sign)
+ * whose fp32 margin is within a guard band of its decision is recomputed in
+ * fp64 before it is stored.
+ *
+ *  layout          d and the bits of this tensor (key_bits if is_key, else
+ *                  value_bits)
+ *  is_key          1: keys (signs + rnorm written, S required); 0: values
+ *  x               device, n_vectors rows of d elements of x_dtype
+ *                  (TQ_F32 or TQ_BF16), row v at x + v*row_stride elements
+ *  positions       device int32 [n_vectors] or NULL
+ *  Pi              device float, row-major d x d matrices; matrix g at
+ *                  Pi + g*pi_stride (pi_stride 0 = one shared matrix)
+ *  vectors_per_pi  rows sharing one Pi (>= 1; ignored when pi_stride == 0)
+ *  S               device float d x d, row-major (keys; NULL for values)
+ *  centroids, boundaries   device float, 2^bits and 2^bits-1 entries
+ *  out             planes to write, n_vectors rows each (pointers device)
+ *  d_status        device int32 (nullable), see TQ_DEV_*
+ * Supported d: 64, 128, 200 (and other multiples of 8 up to 256).
+ * ---------------------------------------------------------------------- */
+tq_status tq_quantize_kv(const tq_layout* layout, int32_t is_key,
+                         const void* x, tq_dtype x_dtype, int64_t n_vectors, int64_t row_stride,
+                         const int32_t* positions, float rope_base,
+                         const float* Pi, int64_t vectors_per_pi, int64_t pi_stride,
+                         const float* S,
+                         const float* centroids, const float* boundaries,
+                         const tq_planes* out,
+                         int32_t* d_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * tq_decode_attention — attention of queries over a packed K/V cache.
+ *
+ * gist.science TurboESM section 2E: one fused kernel unpacks the 3-bit
+ * codes, applies the QJL correction, the inverse rotation Pi^T and an
+ * online-softmax attention, with no dequantised intermediate in memory.
+ * 7minutos.es Etapa 2: the sign bits enter through S^T scaled by
+ * sqrt(pi/2)/d and the residual norm.
+ *
+ * For query row (b, h, n) and its KV head kv = h / (hq/hkv):
+ *   q'    = RoPE(q[b,h,n], q_positions[b*nq + n])   (if enabled)
+ *   q_rot = Pi_K[kv] q',   s = S q_rot
+ *   score_t = scale * ( knorm_t <q_rot, cK[code_t]>
+ *                       + sqrt(pi/2)/d * rnorm_t <s, 2*sign_t - 1> )
+ *   out[b,h,n] = Pi_V[kv]^T sum_t softmax(score)_t vnorm_t cV[vcode_t]
+ * No mask: every query attends all n_ctx tokens.
+ *
+ *  q          device [batch][hq][nq][d] of q_dtype (TQ_F32/TQ_BF16)
+ *  nq         queries per head (1 for decode; up to n_ctx for a full
+ *             bidirectional pass)
+ *  q_positions device int32 [batch][nq] or NULL; rope_base <= 0 disables RoPE
+ *  k, v       planes of [batch][hkv] streams; stream (b, kv) starts at row
+ *             (b*hkv + kv)*ctx_stride; ctx_stride >= n_ctx (0 means n_ctx)
+ *  PiK, PiV   device float d x d; matrix of KV head kv at Pi + kv*pi_stride
+ *             (pi_stride 0 = shared)
+ *  S          device float d x d; cK, cV device centroid tables
+ *  scale      softmax scale (1/sqrt(d) in the method)
+ *  out        device [batch][hq][nq][d] of out_dtype
+ *  scores_out device float [batch][hq][nq][n_ctx] or NULL (raw scores, for
+ *             testing; slows the call)
+ *  workspace  device scratch of tq_decode_workspace_bytes() bytes
+ *             (256-byte aligned); contents need no initialisation
+ * ---------------------------------------------------------------------- */
+tq_status tq_decode_attention(const tq_layout* layout,
+                              const void* q, tq_dtype q_dtype,
+                              int32_t batch, int32_t hq, int32_t hkv, int32_t nq, int64_t n_ctx,
+                              int64_t ctx_stride,
+                              const int32_t* q_positions, float rope_base,
+                              const tq_planes* k, const tq_planes* v,
+                              const float* PiK, const float* PiV, int64_t pi_stride,
+                              const float* S, const float* cK, const float* cV, float scale,
+                              void* out, tq_dtype out_dtype, float* scores_out,
+                              void* workspace, size_t workspace_bytes,
+                              int32_t* d_status, void* stream);
+
+/* Scratch bytes tq_decode_attention needs for this shape (0 on bad args). */
+size_t tq_decode_workspace_bytes(const tq_layout* layout, int32_t batch, int32_t hq, int32_t hkv,
+                                 int32_t nq, int64_t n_ctx);
+
+/* ------------------------------------------------------------------------
+ * tq_dequantize — reconstruct vectors from their planes (device).
+ *
+ * 7minutos.es Etapa 1: look each index up in the codebook and multiply by
+ * the transpose of the rotation, K_hat = Pi^T ||x|| c[code]. Etapa 2:
+ * K_tilde = K_hat + sqrt(pi/2)/d * ||r|| * Pi^T S^T (2*sign - 1)  (keys; S acts
+ * in rotated coordinates, so the correction is turned back by Pi^T too).
+ *
+ *  planes     rows 0..n_vectors-1 (sign/rnorm read only if is_key)
+ *  Pi, vectors_per_pi, pi_stride   as in tq_quantize_kv
+ *  out        device, n_vectors rows of d elements of out_dtype, row v at
+ *             out + v*out_stride elements
+ * ---------------------------------------------------------------------- */
+tq_status tq_dequantize(const tq_layout* layout, int32_t is_key, int64_t n_vectors,
+                        const tq_planes* planes,
+                        const float* Pi, int64_t vectors_per_pi, int64_t pi_stride,
+                        const float* S, const float* centroids,
+                        void* out, tq_dtype out_dtype, int64_t out_stride, void* stream);
+
+/* Description of the last error on this host thread ("" if none). */
+const char* tq_last_error_string(void);
+
+/* Library version string. */
+const char* tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

@@ -1,0 +1,520 @@
+// tq_decode_attention: softmax attention computed directly over the packed
+// K/V planes.
+//
+// Sources: gist.science "TurboESM ..." section 2E (one fused kernel: unpack
+// 3-bit codes, QJL correction, inverse rotation Pi^T, online softmax; no
+// dequantised tensor in memory) and 7minutos.es "KV cache ... TurboQuant"
+// Etapa 2 (sign bits enter through S^T scaled by sqrt(pi/2)/d and ||r||).
+//
+// Three launches on the caller's stream:
+//   1. prologue  q_rot = Pi_K RoPE(q), s = S q_rot for every query row.
+//   2. main      one CTA per (KV stream, query-row block, context split).
+//                Scores use per-CTA shared-memory tables
+//                  Tk[i][c][r] = q_rot[r][i] * cK[c]        (code lookups)
+//                  Ts[i/4][m][r] = sum over 4 coords of +-s (sign nibbles)
+//                so a key costs one table read per coordinate and one per 4
+//                sign bits; V is accumulated in rotated coordinates with an
+//                online softmax; each CTA leaves (m, l, acc) for its split.
+//   3. combine   merges the splits and applies Pi_V^T once per query row.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+using namespace dev;
+
+constexpr int kT = 128;              // tokens per tile = threads of the main kernel
+constexpr int kTargetCtas = 1024;    // split heuristic target (shape-only, device independent)
+constexpr int kMaxRows = 8;          // query rows per main-kernel CTA
+
+struct DecodeShape {
+  int d, kbits, vbits;
+  int batch, hq, hkv, nq;
+  int64_t n_ctx, ctx_stride;
+  int rows_per_cta;   // R
+  int row_blocks;     // (hq/hkv*nq) / R
+  int n_splits;
+  int64_t chunk;      // tokens per split (multiple of kT)
+  int64_t n_rows;     // batch*hq*nq
+};
+
+int pick_rows(int group_rows) {
+  for (int r = kMaxRows; r >= 1; r >>= 1)
+    if (group_rows % r == 0) return r;
+  return 1;
+}
+
+DecodeShape make_shape(const tq_layout* L, int batch, int hq, int hkv, int nq, int64_t n_ctx, int64_t ctx_stride) {
+  DecodeShape s{};
+  s.d = L->d;
+  s.kbits = L->key_bits;
+  s.vbits = L->value_bits;
+  s.batch = batch;
+  s.hq = hq;
+  s.hkv = hkv;
+  s.nq = nq;
+  s.n_ctx = n_ctx;
+  s.ctx_stride = ctx_stride ? ctx_stride : n_ctx;
+  const int group_rows = (hq / hkv) * nq;
+  s.rows_per_cta = pick_rows(group_rows);
+  s.row_blocks = group_rows / s.rows_per_cta;
+  const int64_t units = int64_t(batch) * hkv * s.row_blocks;
+  const int64_t tiles = (n_ctx + kT - 1) / kT;
+  int64_t splits = std::max<int64_t>(1, (kTargetCtas + units - 1) / units);
+  splits = std::min(splits, tiles);
+  const int64_t per = (tiles + splits - 1) / splits;
+  s.chunk = per * kT;
+  s.n_splits = static_cast<int>((n_ctx + s.chunk - 1) / s.chunk);
+  s.n_rows = int64_t(batch) * hq * nq;
+  return s;
+}
+
+size_t shape_workspace_bytes(const DecodeShape& s) {
+  const size_t qs = size_t(s.n_rows) * 2 * s.d * sizeof(float);
+  const size_t part = size_t(s.n_rows) * s.n_splits * (s.d + 2) * sizeof(float);
+  return ((qs + 255) / 256) * 256 + part;
+}
+
+struct DecodeArgs {
+  DecodeShape sh;
+  const void* q;
+  int q_dtype;
+  const int32_t* q_pos;
+  double rope_base;
+  const uint8_t* kidx;
+  const uint32_t* ksign;
+  const float* knorm;
+  const float* krnorm;
+  const uint8_t* vidx;
+  const float* vnorm;
+  const float* PiK;
+  const float* PiV;
+  int64_t pi_stride;
+  const float* S;
+  const float* cK;
+  const float* cV;
+  float scale;
+  void* out;
+  int out_dtype;
+  float* scores_out;
+  float* qs;     // [n_rows][2][d]  q_rot then s
+  float* part;   // [n_rows][n_splits][d + 2]  acc..., m, l
+  int32_t* d_status;
+};
+
+// Query row index -> (b, h, n).
+__device__ __forceinline__ void row_coords(const DecodeShape& s, int64_t row, int& b, int& h, int& n) {
+  n = static_cast<int>(row % s.nq);
+  const int64_t bh = row / s.nq;
+  h = static_cast<int>(bh % s.hq);
+  b = static_cast<int>(bh / s.hq);
+}
+
+// ---------------------------------------------------------------------------
+// 1. Prologue: q_rot = Pi_K[kv] RoPE(q), s = S q_rot (one CTA per query row).
+// ---------------------------------------------------------------------------
+__global__ void decode_prologue(DecodeArgs a) {
+  extern __shared__ double pro_smem[];
+  const DecodeShape& s = a.sh;
+  const int d = s.d;
+  double* qd = pro_smem;            // [d] RoPE'd query
+  float* qr = reinterpret_cast<float*>(pro_smem + d);  // [d] q_rot
+  const int64_t row = blockIdx.x;
+  int b, h, n;
+  row_coords(s, row, b, h, n);
+  const int kv = h / (s.hq / s.hkv);
+  const bool rope = a.q_pos != nullptr && a.rope_base > 0.0;
+  const int pos = rope ? a.q_pos[int64_t(b) * s.nq + n] : 0;
+  if (rope && pos < 0 && threadIdx.x == 0 && a.d_status) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
+  const int64_t qbase = row * d;
+  for (int i = threadIdx.x; i < d / 2; i += blockDim.x) {
+    double x0 = load_elem(a.q, a.q_dtype, qbase + i), x1 = load_elem(a.q, a.q_dtype, qbase + i + d / 2);
+    if (rope) {
+      double sn, cs;
+      sincos(rope_angle(pos, i, d, a.rope_base), &sn, &cs);
+      const double r0 = x0 * cs - x1 * sn, r1 = x0 * sn + x1 * cs;
+      x0 = r0;
+      x1 = r1;
+    }
+    qd[i] = x0;
+    qd[i + d / 2] = x1;
+  }
+  __syncthreads();
+  const float* Pi = a.PiK + kv * a.pi_stride;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    double acc = 0.0;
+    for (int j = 0; j < d; ++j) acc = fma(static_cast<double>(__ldg(Pi + int64_t(i) * d + j)), qd[j], acc);
+    qr[i] = static_cast<float>(acc);
+    a.qs[row * 2 * d + i] = static_cast<float>(acc);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    double acc = 0.0;
+    for (int j = 0; j < d; ++j) acc = fma(static_cast<double>(__ldg(a.S + int64_t(i) * d + j)), double(qr[j]), acc);
+    a.qs[row * 2 * d + d + i] = static_cast<float>(acc);
+  }
+}
+
+// Cooperative byte copy global -> shared with 16-byte vectors when possible.
+__device__ __forceinline__ void stage(void* dst, const void* src, int64_t bytes) {
+  const bool vec = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) | bytes) & 15) == 0;
+  if (vec) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int64_t i = threadIdx.x; i < bytes / 16; i += blockDim.x) d4[i] = __ldg(s4 + i);
+  } else {
+    const uint8_t* s1 = reinterpret_cast<const uint8_t*>(src);
+    uint8_t* d1 = reinterpret_cast<uint8_t*>(dst);
+    for (int64_t i = threadIdx.x; i < bytes; i += blockDim.x) d1[i] = s1[i];
+  }
+}
+
+__device__ __forceinline__ uint32_t group_word(const uint8_t* row, int g, int bits) {
+  const uint8_t* p = row + g * bits;
+  uint32_t w = 0;
+  for (int b = 0; b < bits; ++b) w |= static_cast<uint32_t>(p[b]) << (8 * b);
+  return w;
+}
+
+// ---------------------------------------------------------------------------
+// 2. Main split-KV kernel.
+// ---------------------------------------------------------------------------
+template <int D, int R>
+struct MainSmem {
+  static constexpr int kSW = (D + 31) / 32;
+  float sc[kT][R];           // scores of the tile
+  float w[kT][R];            // exp(score - m) * ||v||
+  float knorm[kT], krn[kT], vnorm[kT];
+  uint32_t ksign[kT][kSW];
+  float red[kT / kWarp][R];
+  float m[R], l[R], corr[R];
+  float cV[16];
+  // followed by: Tk[D][nck][R], Ts[D/4][16][R], kidx[kT*rbk], vidx[kT*rbv]
+};
+
+template <int D, int R>
+__global__ void __launch_bounds__(kT) decode_main(DecodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  using Sm = MainSmem<D, R>;
+  Sm& s = *reinterpret_cast<Sm*>(smem_raw);
+  const DecodeShape& sh = a.sh;
+  const int nck = 1 << sh.kbits, ncv = 1 << sh.vbits;
+  const int rbk = D * sh.kbits / 8, rbv = D * sh.vbits / 8;
+  float* Tk = reinterpret_cast<float*>(smem_raw + ((sizeof(Sm) + 15) / 16) * 16);
+  float* Ts = Tk + D * nck * R;
+  uint8_t* kidx = reinterpret_cast<uint8_t*>(Ts + (D / 4) * 16 * R);
+  uint8_t* vidx = kidx + ((kT * rbk + 15) / 16) * 16;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x;
+  const int64_t unit = blockIdx.y;                      // (b, kv, row block)
+  const int rb = static_cast<int>(unit % sh.row_blocks);
+  const int64_t bkv = unit / sh.row_blocks;             // b*hkv + kv
+  const int G = sh.hq / sh.hkv;
+  const int kv = static_cast<int>(bkv % sh.hkv);
+  const int b = static_cast<int>(bkv / sh.hkv);
+  // Query row r of this CTA: group-local index rr = rb*R + r -> head kv*G + rr/nq, query rr%nq.
+  auto qrow = [&](int r) -> int64_t {
+    const int rr = rb * R + r;
+    const int h = kv * G + rr / sh.nq;
+    return (int64_t(b) * sh.hq + h) * sh.nq + rr % sh.nq;
+  };
+
+  // Tables.
+  if (tid < ncv) s.cV[tid] = a.cV[tid];
+  for (int e = tid; e < D * nck * R; e += kT) {
+    const int r = e % R, c = (e / R) % nck, i = e / (R * nck);
+    Tk[e] = a.qs[qrow(r) * 2 * D + i] * __ldg(a.cK + c);
+  }
+  for (int e = tid; e < (D / 4) * 16 * R; e += kT) {
+    const int r = e % R, m = (e / R) % 16, nib = e / (R * 16);
+    const float* sv = a.qs + qrow(r) * 2 * D + D + 4 * nib;
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc += ((m >> q) & 1) ? sv[q] : -sv[q];
+    Ts[e] = acc;
+  }
+  if (tid < R) {
+    s.m[tid] = -INFINITY;
+    s.l[tid] = 0.f;
+  }
+  float acc[(D + kT - 1) / kT][R];
+#pragma unroll
+  for (int c = 0; c < (D + kT - 1) / kT; ++c)
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[c][r] = 0.f;
+
+  const float alpha = static_cast<float>(kSqrtHalfPi / D);
+  const int64_t t_begin = int64_t(split) * sh.chunk;
+  const int64_t t_end = (t_begin + sh.chunk < sh.n_ctx) ? t_begin + sh.chunk : sh.n_ctx;
+  const int64_t row0 = bkv * sh.ctx_stride;
+
+  for (int64_t t0 = t_begin; t0 < t_end; t0 += kT) {
+    const int nt = static_cast<int>((t_end - t0 < kT) ? t_end - t0 : kT);
+    __syncthreads();
+    stage(kidx, a.kidx + (row0 + t0) * rbk, int64_t(nt) * rbk);
+    stage(vidx, a.vidx + (row0 + t0) * rbv, int64_t(nt) * rbv);
+    stage(&s.ksign[0][0], a.ksign + (row0 + t0) * Sm::kSW, int64_t(nt) * Sm::kSW * 4);
+    if (tid < nt) {
+      s.knorm[tid] = __ldg(a.knorm + row0 + t0 + tid);
+      s.krn[tid] = __ldg(a.krnorm + row0 + t0 + tid);
+      s.vnorm[tid] = __ldg(a.vnorm + row0 + t0 + tid);
+    }
+    __syncthreads();
+
+    // Scores: thread = token.
+    float score[R];
+    if (tid < nt) {
+      float ck[R], cs[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) ck[r] = cs[r] = 0.f;
+      const uint8_t* row = kidx + tid * rbk;
+      for (int g = 0; g < D / 8; ++g) {
+        const uint32_t word = group_word(row, g, sh.kbits);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = (word >> (sh.kbits * j)) & (nck - 1);
+          const float* e = Tk + ((8 * g + j) * nck + c) * R;
+#pragma unroll
+          for (int r = 0; r < R; ++r) ck[r] += e[r];
+        }
+      }
+      for (int nib = 0; nib < D / 4; ++nib) {
+        const int m = (s.ksign[tid][nib >> 3] >> (4 * (nib & 7))) & 15;
+        const float* e = Ts + (nib * 16 + m) * R;
+#pragma unroll
+        for (int r = 0; r < R; ++r) cs[r] += e[r];
+      }
+      const float kn = s.knorm[tid], rn = s.krn[tid];
+#pragma unroll
+      for (int r = 0; r < R; ++r) score[r] = a.scale * (kn * ck[r] + alpha * rn * cs[r]);
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r) score[r] = -INFINITY;
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) s.sc[tid][r] = score[r];
+    if (a.scores_out && tid < nt) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) a.scores_out[qrow(r) * sh.n_ctx + t0 + tid] = score[r];
+    }
+    // Tile max per row.
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float mx = warp_max(score[r]);
+      if (lane == 0) s.red[warp][r] = mx;
+    }
+    __syncthreads();
+    if (tid < R) {
+      float mx = s.red[0][tid];
+      for (int w2 = 1; w2 < kT / kWarp; ++w2) mx = fmaxf(mx, s.red[w2][tid]);
+      const float m_new = fmaxf(s.m[tid], mx);
+      s.corr[tid] = (s.m[tid] == -INFINITY) ? 0.f : expf(s.m[tid] - m_new);
+      s.m[tid] = m_new;
+    }
+    __syncthreads();
+    float psum[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float p = (tid < nt) ? expf(score[r] - s.m[r]) : 0.f;
+      s.w[tid][r] = p * ((tid < nt) ? s.vnorm[tid] : 0.f);
+      psum[r] = warp_sum(p);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (lane == 0) s.red[warp][r] = psum[r];
+    __syncthreads();
+    if (tid < R) {
+      float tot = 0.f;
+      for (int w2 = 0; w2 < kT / kWarp; ++w2) tot += s.red[w2][tid];
+      s.l[tid] = s.l[tid] * s.corr[tid] + tot;
+    }
+    // V: thread = coordinate.
+#pragma unroll
+    for (int c = 0; c < (D + kT - 1) / kT; ++c) {
+      const int i = tid + c * kT;
+      if (i < D) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[c][r] *= s.corr[r];
+        for (int t = 0; t < nt; ++t) {
+          const float cv = s.cV[get_code(vidx + t * rbv, i, sh.vbits)];
+#pragma unroll
+          for (int r = 0; r < R; ++r) acc[c][r] = fmaf(s.w[t][r], cv, acc[c][r]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // Partials.
+#pragma unroll
+  for (int c = 0; c < (D + kT - 1) / kT; ++c) {
+    const int i = tid + c * kT;
+    if (i < D) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) a.part[(qrow(r) * sh.n_splits + split) * (D + 2) + i] = acc[c][r];
+    }
+  }
+  if (tid < R) {
+    float* p = a.part + (qrow(tid) * sh.n_splits + split) * (D + 2);
+    p[D] = s.m[tid];
+    p[D + 1] = s.l[tid];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. Combine the splits and turn back by Pi_V^T (one CTA per query row).
+// ---------------------------------------------------------------------------
+__global__ void decode_combine(DecodeArgs a) {
+  extern __shared__ float cmb[];
+  const DecodeShape& s = a.sh;
+  const int d = s.d;
+  const int64_t row = blockIdx.x;
+  int b, h, n;
+  row_coords(s, row, b, h, n);
+  const int kv = h / (s.hq / s.hkv);
+  const float* part = a.part + row * s.n_splits * (d + 2);
+  float M = -INFINITY;
+  for (int k = 0; k < s.n_splits; ++k) M = fmaxf(M, part[k * (d + 2) + d]);
+  float L = 0.f;
+  for (int k = 0; k < s.n_splits; ++k) {
+    const float mk = part[k * (d + 2) + d];
+    if (mk > -INFINITY) L += expf(mk - M) * part[k * (d + 2) + d + 1];
+  }
+  float* o = cmb;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float acc = 0.f;
+    for (int k = 0; k < s.n_splits; ++k) {
+      const float mk = part[k * (d + 2) + d];
+      if (mk > -INFINITY) acc += expf(mk - M) * part[k * (d + 2) + i];
+    }
+    o[i] = acc / L;
+  }
+  __syncthreads();
+  const float* Pi = a.PiV + kv * a.pi_stride;
+  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < d; ++i) acc = fmaf(__ldg(Pi + int64_t(i) * d + j), o[i], acc);
+    if (a.out_dtype == 0)
+      reinterpret_cast<float*>(a.out)[row * d + j] = acc;
+    else
+      reinterpret_cast<__nv_bfloat16*>(a.out)[row * d + j] = __float2bfloat16(acc);
+  }
+}
+
+template <int D, int R>
+cudaError_t launch_main(const DecodeArgs& a, cudaStream_t st) {
+  using Sm = MainSmem<D, R>;
+  const int nck = 1 << a.sh.kbits;
+  const int rbk = D * a.sh.kbits / 8, rbv = D * a.sh.vbits / 8;
+  const size_t smem = ((sizeof(Sm) + 15) / 16) * 16 + sizeof(float) * (D * nck * R + (D / 4) * 16 * R) +
+                      ((kT * rbk + 15) / 16) * 16 + ((kT * rbv + 15) / 16) * 16;
+  cudaError_t e = cudaFuncSetAttribute(decode_main<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.sh.n_splits, static_cast<unsigned>(int64_t(a.sh.batch) * a.sh.hkv * a.sh.row_blocks));
+  decode_main<D, R><<<grid, kT, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_main_rows(const DecodeArgs& a, cudaStream_t st) {
+  switch (a.sh.rows_per_cta) {
+    case 1: return launch_main<D, 1>(a, st);
+    case 2: return launch_main<D, 2>(a, st);
+    case 4: return launch_main<D, 4>(a, st);
+    default: return launch_main<D, 8>(a, st);
+  }
+}
+
+}  // namespace
+}  // namespace tq
+
+extern "C" size_t tq_decode_workspace_bytes(const tq_layout* layout, int32_t batch, int32_t hq, int32_t hkv,
+                                            int32_t nq, int64_t n_ctx) {
+  if (tq::check_layout(layout) != TQ_OK || batch < 1 || hkv < 1 || hq < hkv || hq % hkv || nq < 1 || n_ctx < 1)
+    return 0;
+  return tq::shape_workspace_bytes(tq::make_shape(layout, batch, hq, hkv, nq, n_ctx, n_ctx));
+}
+
+extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q, tq_dtype q_dtype, int32_t batch,
+                                         int32_t hq, int32_t hkv, int32_t nq, int64_t n_ctx, int64_t ctx_stride,
+                                         const int32_t* q_positions, float rope_base, const tq_planes* k,
+                                         const tq_planes* v, const float* PiK, const float* PiV, int64_t pi_stride,
+                                         const float* S, const float* cK, const float* cV, float scale, void* out,
+                                         tq_dtype out_dtype, float* scores_out, void* workspace,
+                                         size_t workspace_bytes, int32_t* d_status, void* stream) {
+  using namespace tq;
+  clear_error();
+  tq_status st = check_layout(layout);
+  if (st != TQ_OK) return st;
+  const int d = layout->d;
+  if (batch < 1 || hkv < 1 || hq < hkv || hq % hkv != 0 || nq < 1)
+    return fail(TQ_ERR_INVALID_ARG, "need batch>=1, hkv>=1, hq a multiple of hkv, nq>=1");
+  if (n_ctx < 1) return fail(TQ_ERR_INVALID_ARG, "n_ctx must be >= 1 (softmax over an empty cache is undefined)");
+  if (ctx_stride != 0 && ctx_stride < n_ctx) return fail(TQ_ERR_INVALID_ARG, "ctx_stride < n_ctx");
+  if (!q || !k || !v || !k->idx || !k->sign || !k->norm || !k->rnorm || !v->idx || !v->norm || !PiK || !PiV || !S ||
+      !cK || !cV || !out)
+    return fail(TQ_ERR_INVALID_ARG, "NULL pointer argument");
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_F32 or TQ_BF16");
+  if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return fail(TQ_ERR_INVALID_ARG, "out_dtype must be TQ_F32 or TQ_BF16");
+  if (pi_stride < 0) return fail(TQ_ERR_INVALID_ARG, "pi_stride < 0");
+  if (!aligned(k->idx, 16) || !aligned(k->sign, 16) || !aligned(v->idx, 16))
+    return fail(TQ_ERR_INVALID_ARG, "plane pointers must be 16-byte aligned");
+  const DecodeShape sh = make_shape(layout, batch, hq, hkv, nq, n_ctx, ctx_stride);
+  const size_t need = shape_workspace_bytes(sh);
+  if (!workspace || workspace_bytes < need)
+    return fail(TQ_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (sh.n_rows > (int64_t(1) << 31) - 1 || int64_t(batch) * hkv * sh.row_blocks > 65535)
+    return fail(TQ_ERR_UNSUPPORTED, "too many query rows / KV streams for one call");
+  DecodeArgs a{};
+  a.sh = sh;
+  a.q = q;
+  a.q_dtype = q_dtype == TQ_F32 ? 0 : 1;
+  a.q_pos = q_positions;
+  a.rope_base = rope_base;
+  a.kidx = k->idx;
+  a.ksign = k->sign;
+  a.knorm = k->norm;
+  a.krnorm = k->rnorm;
+  a.vidx = v->idx;
+  a.vnorm = v->norm;
+  a.PiK = PiK;
+  a.PiV = PiV;
+  a.pi_stride = pi_stride;
+  a.S = S;
+  a.cK = cK;
+  a.cV = cV;
+  a.scale = scale;
+  a.out = out;
+  a.out_dtype = out_dtype == TQ_F32 ? 0 : 1;
+  a.scores_out = scores_out;
+  a.qs = static_cast<float*>(workspace);
+  a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                    ((size_t(sh.n_rows) * 2 * d * sizeof(float) + 255) / 256) * 256);
+  a.d_status = d_status;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  decode_prologue<<<static_cast<unsigned>(sh.n_rows), 128, (d * sizeof(double) + d * sizeof(float)), s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {
+    switch (d) {
+      case 64: e = launch_main_rows<64>(a, s); break;
+      case 128: e = launch_main_rows<128>(a, s); break;
+      case 200: e = launch_main_rows<200>(a, s); break;
+      default: return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: d=%d not built (64, 128, 200)", d);
+    }
+  }
+  if (e == cudaSuccess) {
+    decode_combine<<<static_cast<unsigned>(sh.n_rows), 128, d * sizeof(float), s>>>(a);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_decode_attention launch: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}

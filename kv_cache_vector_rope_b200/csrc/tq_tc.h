@@ -1,0 +1,19 @@
+// Internal interface of the tensor-core quantiser (tq_quantize_tc.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tq.h"
+
+namespace tq {
+
+// True when the tensor-core path applies: d 64 or 128, bf16 input rows with
+// 16-byte aligned base and stride, no RoPE, one shared Pi.
+bool tc_quantize_supported(int d, int x_dtype, bool rope, int64_t pi_stride, const void* x, int64_t row_stride);
+
+tq_status tc_quantize(int d, bool is_key, int bits, const void* x, int64_t n, int64_t row_stride, const float* Pi,
+                      const float* S, const float* cent, const float* bnd, const tq_planes* out, int32_t* d_status,
+                      cudaStream_t st);
+
+}  // namespace tq
