@@ -233,6 +233,33 @@ tq_status tq_dequantize(const tq_layout* layout, int32_t is_key, int64_t n_vecto
                         const float* S, const float* centroids,
                         void* out, tq_dtype out_dtype, int64_t out_stride, void* stream);
 
+/* ------------------------------------------------------------------------
+ * tq_fit_rotation — per-head rotation from calibration vectors (host only).
+ *
+ * gist.science TurboESM section 2B: instead of one global or random matrix,
+ * a Pi is computed for every layer and attention head by SVD of real
+ * activations, equalising the variance across directions.
+ *
+ *   X        host float [n][d]: the head's calibration vectors (uncentred)
+ *   Pi_rand  host float [d][d]: the seeded random rotation
+ *   Pi_out   host float [d][d]: Pi_rand V^T, V the right singular vectors of
+ *            X (decreasing singular value; each signed so its largest-magnitude
+ *            entry is positive)
+ * Computed in fp64 (cyclic Jacobi on X^T X). Errors: TQ_ERR_INVALID_ARG.
+ * ---------------------------------------------------------------------- */
+tq_status tq_fit_rotation(int32_t d, const float* X, int64_t n, const float* Pi_rand, float* Pi_out);
+
+/* ------------------------------------------------------------------------
+ * tq_rotate_normalize — samples for the dual (K / V) codebooks (host only).
+ *
+ * gist.science TurboESM section 2C: K and V tables are fitted to their own
+ * post-rotation coordinate distributions. Writes the coordinates of
+ * Pi x / ||x|| for every non-zero row x of X (rows in order; zero rows have no
+ * direction and are skipped) to u_out [n_out][d], fp64 internally.
+ * Feed the pooled samples to tq_make_codebook(mode = 1).
+ * ---------------------------------------------------------------------- */
+tq_status tq_rotate_normalize(int32_t d, const float* X, int64_t n, const float* Pi, float* u_out, int64_t* n_out);
+
 /* Description of the last error on this host thread ("" if none). */
 const char* tq_last_error_string(void);
 

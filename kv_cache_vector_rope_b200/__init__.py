@@ -61,6 +61,8 @@ _SIGNATURES = {
     "tq_decode_workspace_bytes": (_SZ, [ctypes.POINTER(Layout), _I32, _I32, _I32, _I32, _I64]),
     "tq_dequantize": (ctypes.c_int, [ctypes.POINTER(Layout), _I32, _I64, ctypes.POINTER(_Planes), _P, _I64, _I64,
                                      _P, _P, _P, ctypes.c_int, _I64, _P]),
+    "tq_fit_rotation": (ctypes.c_int, [_I32, _P, _I64, _P, _P]),
+    "tq_rotate_normalize": (ctypes.c_int, [_I32, _P, _I64, _P, _P, ctypes.POINTER(_I64)]),
     "tq_last_error_string": (ctypes.c_char_p, []),
     "tq_version": (ctypes.c_char_p, []),
 }
@@ -68,7 +70,7 @@ _SIGNATURES = {
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libtq.so is not built ({LIB_PATH}); run `python -m kv_cache_vector_rope_b200.build` "
+        raise ImportError(f"libtq.so is not built ({LIB_PATH}); run `python kv_cache_vector_rope_b200/build.py` "
                           "(the CUDA library is the only implementation; there is no fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():
@@ -235,6 +237,27 @@ def tq_dequantize(lay: Layout, is_key: bool, planes: Planes, n_vectors: int, Pi:
     _check(_lib.tq_dequantize(ctypes.byref(lay), int(is_key), n_vectors, ctypes.byref(planes.c()),
                               _dev(Pi, "Pi"), vectors_per_pi, pi_stride, _ptr(S), _dev(centroids, "centroids"),
                               _dev(out, "out"), _dtype_code(out), out.stride(0), _stream(stream)))
+
+
+def tq_fit_rotation(X, Pi_rand) -> np.ndarray:
+    """Per-head rotation Pi_rand V^T from calibration rows X ([n, d], host)."""
+    X = np.ascontiguousarray(np.asarray(X, dtype=np.float32))
+    P = np.ascontiguousarray(np.asarray(Pi_rand, dtype=np.float32))
+    n, d = X.shape
+    out = np.zeros((d, d), dtype=np.float32)
+    _check(_lib.tq_fit_rotation(d, X.ctypes.data, n, P.ctypes.data, out.ctypes.data))
+    return out
+
+
+def tq_rotate_normalize(X, Pi) -> np.ndarray:
+    """Coordinates of Pi x / ||x|| for the non-zero rows of X (host)."""
+    X = np.ascontiguousarray(np.asarray(X, dtype=np.float32))
+    P = np.ascontiguousarray(np.asarray(Pi, dtype=np.float32))
+    n, d = X.shape
+    out = np.zeros((n, d), dtype=np.float32)
+    m = ctypes.c_int64(0)
+    _check(_lib.tq_rotate_normalize(d, X.ctypes.data, n, P.ctypes.data, out.ctypes.data, ctypes.byref(m)))
+    return out[:m.value]
 
 
 def tq_last_error_string() -> str:

@@ -1,7 +1,10 @@
 """Builds libtq.so (the CUDA library behind the C ABI in include/tq.h) in-tree.
 
-    python -m kv_cache_vector_rope_b200.build          # compile if stale
-    python -m kv_cache_vector_rope_b200.build --force  # always compile
+    python kv_cache_vector_rope_b200/build.py          # compile if stale
+    python kv_cache_vector_rope_b200/build.py --force  # always compile
+
+Runs as a plain script (it must not import the package, whose binding loads
+the library being built).
 
 Everything is compiled for sm_100a only (B200).
 """

@@ -49,7 +49,6 @@ using namespace sm100;
 using dev::warp_sum;
 
 constexpr int kThreads = 320;         // 10 warps
-constexpr int kEpiThreads = 256;      // warps 2..9
 // Guard bands. The fp32 accumulation of the 3-way split rotation errs by
 // ~1e-7 ||x|| per coordinate (std), the 2x2-way split projection by ~3e-6 ||r||,
 // and the fp32 residual moves an fp64 projection by ~5e-7 ||r||: each band is
@@ -425,7 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       const float band = kCodeGuard * nrm;
 #pragma unroll
       for (int j = 0; j < kNb; ++j) th[j] = nrm * bnd_s[j];
-      const __nv_bfloat16* xrow = a.x + (valid ? v : 0) * a.row_stride;
 
       uint32_t codew[C::kChunksPerWg][BITS];
       float rsq = 0.f;

@@ -159,3 +159,38 @@ def test_dequantize_host_validation():
     assert f(ctypes.byref(lay), 0, 10, ctypes.byref(p), 0x5000, 1, 0, None, 0x6000, 0x7000, 0, 64, None) \
         == tq.TQ_ERR_INVALID_ARG     # out_stride < d
     assert f(ctypes.byref(lay), 0, 0, ctypes.byref(p), 0x5000, 1, 0, None, 0x6000, 0x7000, 0, 128, None) == tq.TQ_OK
+
+
+def test_fit_rotation_matches_oracle_svd_basis():
+    from oracle import calib as oc
+    import synth
+    rg = np.random.default_rng(41)
+    for d in (64, 128):
+        X = rg.standard_normal((256, d))
+        X[:, rg.choice(d, 4, replace=False)] *= rg.lognormal(2.0, 1.0, 4)
+        X32 = X.astype(np.float32)
+        Pr = synth.random_rotation(d, 5)
+        got = tq.tq_fit_rotation(X32, Pr)
+        ref = oc.head_rotation(Pr, X32.astype(np.float64))
+        np.testing.assert_allclose(got, ref, atol=2e-6)
+        np.testing.assert_allclose(got.astype(np.float64).T @ got, np.eye(d), atol=5e-6)
+
+
+def test_rotate_normalize_matches_oracle_and_skips_zero_rows():
+    from oracle import calib as oc
+    import synth
+    rg = np.random.default_rng(42)
+    X = rg.standard_normal((50, 64)).astype(np.float32)
+    X[7] = 0.0
+    P = synth.random_rotation(64, 1)
+    got = tq.tq_rotate_normalize(X, P)
+    assert got.shape == (49, 64)
+    ref = oc.rotated_unit_coordinates(X.astype(np.float64), P).reshape(-1, 64)
+    np.testing.assert_allclose(got, ref, atol=1e-7)
+
+
+def test_calibration_argument_errors():
+    with pytest.raises(tq.TQError):
+        tq.tq_fit_rotation(np.zeros((0, 64), np.float32), np.eye(64, dtype=np.float32))
+    with pytest.raises(tq.TQError):
+        tq.tq_fit_rotation(np.full((4, 64), np.nan, np.float32), np.eye(64, dtype=np.float32))
