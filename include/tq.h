@@ -234,6 +234,32 @@ tq_status tq_dequantize(const tq_layout* layout, int32_t is_key, int64_t n_vecto
                         void* out, tq_dtype out_dtype, int64_t out_stride, void* stream);
 
 /* ------------------------------------------------------------------------
+ * tq_search_topk — k best corpus vectors per query by estimated inner product.
+ *
+ * sudonull.com "TurboQuant: compresión 6x de LLM KV-cache" and news.hada.io's
+ * TurboQuant summary: the same codes serve vector search (recall of the true
+ * top inner products among the approximate top-k). Score of corpus vector x
+ * (quantised as a key: codes, signs, ||x||, ||r||) for query q:
+ *   est = ||x|| <Pi q, c[code_x]> + sqrt(pi/2)/d ||r_x|| <S Pi q, 2 sign_x - 1>
+ * Ranking: decreasing est; equal scores by increasing corpus index.
+ *
+ *  q           device [n_queries][d] of q_dtype
+ *  db          key planes of n_db corpus vectors (layout.key_bits bits)
+ *  Pi, S       device float d x d (the ones the corpus was quantised with)
+ *  centroids   device float, 2^key_bits entries
+ *  k           1..32 (and <= n_db)
+ *  top_idx     device int64 [n_queries][k], top_scores device float [n_queries][k]
+ *  workspace   device scratch of tq_search_workspace_bytes() (256-B aligned)
+ * ---------------------------------------------------------------------- */
+tq_status tq_search_topk(const tq_layout* layout, const void* q, tq_dtype q_dtype, int32_t n_queries,
+                         const tq_planes* db, int64_t n_db, const float* Pi, const float* S,
+                         const float* centroids, int32_t k, int64_t* top_idx, float* top_scores,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Scratch bytes tq_search_topk needs (0 on invalid arguments). */
+size_t tq_search_workspace_bytes(const tq_layout* layout, int32_t n_queries, int64_t n_db, int32_t k);
+
+/* ------------------------------------------------------------------------
  * tq_fit_rotation — per-head rotation from calibration vectors (host only).
  *
  * gist.science TurboESM section 2B: instead of one global or random matrix,

@@ -61,6 +61,9 @@ _SIGNATURES = {
     "tq_decode_workspace_bytes": (_SZ, [ctypes.POINTER(Layout), _I32, _I32, _I32, _I32, _I64]),
     "tq_dequantize": (ctypes.c_int, [ctypes.POINTER(Layout), _I32, _I64, ctypes.POINTER(_Planes), _P, _I64, _I64,
                                      _P, _P, _P, ctypes.c_int, _I64, _P]),
+    "tq_search_topk": (ctypes.c_int, [ctypes.POINTER(Layout), _P, ctypes.c_int, _I32, ctypes.POINTER(_Planes), _I64,
+                                      _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
+    "tq_search_workspace_bytes": (_SZ, [ctypes.POINTER(Layout), _I32, _I64, _I32]),
     "tq_fit_rotation": (ctypes.c_int, [_I32, _P, _I64, _P, _P]),
     "tq_rotate_normalize": (ctypes.c_int, [_I32, _P, _I64, _P, _P, ctypes.POINTER(_I64)]),
     "tq_last_error_string": (ctypes.c_char_p, []),
@@ -237,6 +240,22 @@ def tq_dequantize(lay: Layout, is_key: bool, planes: Planes, n_vectors: int, Pi:
     _check(_lib.tq_dequantize(ctypes.byref(lay), int(is_key), n_vectors, ctypes.byref(planes.c()),
                               _dev(Pi, "Pi"), vectors_per_pi, pi_stride, _ptr(S), _dev(centroids, "centroids"),
                               _dev(out, "out"), _dtype_code(out), out.stride(0), _stream(stream)))
+
+
+def tq_search_workspace_bytes(lay: Layout, n_queries: int, n_db: int, k: int) -> int:
+    return int(_lib.tq_search_workspace_bytes(ctypes.byref(lay), n_queries, n_db, k))
+
+
+def tq_search_topk(lay: Layout, q: torch.Tensor, db: Planes, n_db: int, Pi: torch.Tensor, S: torch.Tensor,
+                   centroids: torch.Tensor, k: int, top_idx: torch.Tensor, top_scores: torch.Tensor,
+                   workspace: torch.Tensor, stream=None) -> None:
+    """k best corpus rows per query ([n_queries, d], contiguous) by estimated inner product."""
+    if q.dim() != 2 or not q.is_contiguous():
+        raise ValueError("q must be a contiguous [n_queries, d] tensor")
+    _check(_lib.tq_search_topk(ctypes.byref(lay), _dev(q, "q"), _dtype_code(q), q.shape[0], ctypes.byref(db.c()),
+                               n_db, _dev(Pi, "Pi"), _dev(S, "S"), _dev(centroids, "centroids"), k,
+                               _dev(top_idx, "top_idx"), _dev(top_scores, "top_scores"), _dev(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def tq_fit_rotation(X, Pi_rand) -> np.ndarray:
