@@ -21,6 +21,8 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
@@ -408,6 +410,38 @@ __global__ void decode_combine(DecodeArgs a) {
   }
 }
 
+}  // namespace
+}  // namespace tq
+
+#include "tq_decode_v2.cuh"
+
+namespace tq {
+namespace {
+
+template <int D, int R, int KB>
+cudaError_t launch_v2(const DecodeArgs& a, cudaStream_t st) {
+  using Sm = V2Smem<D, R, KB>;
+  cudaError_t e = cudaFuncSetAttribute(decode_main_v2<D, R, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.sh.n_splits, static_cast<unsigned>(int64_t(a.sh.batch) * a.sh.hkv * a.sh.row_blocks));
+  decode_main_v2<D, R, KB><<<grid, kT2, Sm::kBytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+// Version-2 kernel when it applies: d 64/128, 4 or 8 query rows per CTA,
+// 3-bit values. Returns false to fall back to the general kernel.
+template <int D>
+bool try_v2(const DecodeArgs& a, cudaStream_t st, cudaError_t& e) {
+  if (a.sh.vbits != 3 || !(a.sh.rows_per_cta == 4 || a.sh.rows_per_cta == 8)) return false;
+  const bool r4 = a.sh.rows_per_cta == 4;
+  switch (a.sh.kbits) {
+    case 2: e = r4 ? launch_v2<D, 4, 2>(a, st) : launch_v2<D, 8, 2>(a, st); return true;
+    case 3: e = r4 ? launch_v2<D, 4, 3>(a, st) : launch_v2<D, 8, 3>(a, st); return true;
+    case 4: e = r4 ? launch_v2<D, 4, 4>(a, st) : launch_v2<D, 8, 4>(a, st); return true;
+    default: return false;
+  }
+}
+
 template <int D, int R>
 cudaError_t launch_main(const DecodeArgs& a, cudaStream_t st) {
   using Sm = MainSmem<D, R>;
@@ -425,6 +459,13 @@ cudaError_t launch_main(const DecodeArgs& a, cudaStream_t st) {
 
 template <int D>
 cudaError_t launch_main_rows(const DecodeArgs& a, cudaStream_t st) {
+  if (D == 64 || D == 128) {
+    const char* env = std::getenv("TQ_DECODE_PATH");
+    if (!(env && std::strcmp(env, "v1") == 0)) {
+      cudaError_t e = cudaSuccess;
+      if (try_v2<(D == 64 ? 64 : 128)>(a, st, e)) return e;
+    }
+  }
   switch (a.sh.rows_per_cta) {
     case 1: return launch_main<D, 1>(a, st);
     case 2: return launch_main<D, 2>(a, st);
