@@ -215,6 +215,37 @@ size_t tq_decode_workspace_bytes(const tq_layout* layout, int32_t batch, int32_t
                                  int32_t nq, int64_t n_ctx);
 
 /* ------------------------------------------------------------------------
+ * tq_decode_attention_noalloc — tq_decode_attention without a caller
+ * workspace. (No counterpart in the method's description; it exists for
+ * callers that cannot allocate device memory at call time — a serving loop
+ * that must not stall on cudaMalloc's implicit device synchronisation, or a
+ * plugin inside a host framework that owns every device allocation.)
+ *
+ * Arguments and results are those of tq_decode_attention minus
+ * workspace/workspace_bytes. The split-KV scratch is a fixed 64 MiB device
+ * array inside libtq.so (every GPU that loads the library holds it until the
+ * process exits); shapes whose tq_decode_workspace_bytes() exceeds 64 MiB are
+ * rejected with TQ_ERR_UNSUPPORTED and a message. The function itself calls
+ * no cudaMalloc/cudaFree and no allocating routine.
+ *  - The first call on each device looks the array's device address up
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and leave their data in it. Nothing needs
+ *    clearing between calls, but calls that overlap on the GPU (other streams
+ *    or host threads) race on it: serialise them.
+ * ---------------------------------------------------------------------- */
+tq_status tq_decode_attention_noalloc(const tq_layout* layout,
+                                      const void* q, tq_dtype q_dtype,
+                                      int32_t batch, int32_t hq, int32_t hkv, int32_t nq, int64_t n_ctx,
+                                      int64_t ctx_stride,
+                                      const int32_t* q_positions, float rope_base,
+                                      const tq_planes* k, const tq_planes* v,
+                                      const float* PiK, const float* PiV, int64_t pi_stride,
+                                      const float* S, const float* cK, const float* cV, float scale,
+                                      void* out, tq_dtype out_dtype, float* scores_out,
+                                      int32_t* d_status, void* stream);
+
+/* ------------------------------------------------------------------------
  * tq_dequantize — reconstruct vectors from their planes (device).
  *
  * 7minutos.es Etapa 1: look each index up in the codebook and multiply by

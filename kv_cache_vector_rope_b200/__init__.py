@@ -59,6 +59,10 @@ _SIGNATURES = {
                                            _I64, _P, _F32, ctypes.POINTER(_Planes), ctypes.POINTER(_Planes),
                                            _P, _P, _I64, _P, _P, _P, _F32, _P, ctypes.c_int, _P, _P, _SZ, _P, _P]),
     "tq_decode_workspace_bytes": (_SZ, [ctypes.POINTER(Layout), _I32, _I32, _I32, _I32, _I64]),
+    "tq_decode_attention_noalloc": (ctypes.c_int, [ctypes.POINTER(Layout), _P, ctypes.c_int, _I32, _I32, _I32, _I32,
+                                                   _I64, _I64, _P, _F32, ctypes.POINTER(_Planes),
+                                                   ctypes.POINTER(_Planes), _P, _P, _I64, _P, _P, _P, _F32, _P,
+                                                   ctypes.c_int, _P, _P, _P]),
     "tq_dequantize": (ctypes.c_int, [ctypes.POINTER(Layout), _I32, _I64, ctypes.POINTER(_Planes), _P, _I64, _I64,
                                      _P, _P, _P, ctypes.c_int, _I64, _P]),
     "tq_search_topk": (ctypes.c_int, [ctypes.POINTER(Layout), _P, ctypes.c_int, _I32, ctypes.POINTER(_Planes), _I64,
@@ -230,6 +234,28 @@ def tq_decode_attention(lay: Layout, q: torch.Tensor, k: Planes, v: Planes, hkv:
         _dev(PiK, "PiK"), _dev(PiV, "PiV"), pi_stride, _dev(S, "S"), _dev(cK, "cK"), _dev(cV, "cV"),
         float(scale), _dev(out, "out"), _dtype_code(out), _ptr(scores_out), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _ptr(d_status), _stream(stream)))
+
+
+def tq_decode_attention_noalloc(lay: Layout, q: torch.Tensor, k: Planes, v: Planes, hkv: int, n_ctx: int,
+                                PiK: torch.Tensor, PiV: torch.Tensor, S: torch.Tensor, cK: torch.Tensor,
+                                cV: torch.Tensor, out: torch.Tensor, scale: float | None = None,
+                                q_positions: torch.Tensor | None = None, rope_base: float = 0.0, pi_stride: int = 0,
+                                ctx_stride: int = 0, scores_out: torch.Tensor | None = None,
+                                d_status: torch.Tensor | None = None, stream=None) -> None:
+    """tq_decode_attention with the library's fixed device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory at call time. Calls that
+    overlap on the GPU share the scratch and must be serialised by the caller."""
+    if q.dim() != 4 or not q.is_contiguous() or not out.is_contiguous():
+        raise ValueError("q and out must be contiguous [batch, hq, nq, d] tensors")
+    batch, hq, nq, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    _check(_lib.tq_decode_attention_noalloc(
+        ctypes.byref(lay), _dev(q, "q"), _dtype_code(q), batch, hq, hkv, nq, n_ctx, ctx_stride,
+        _ptr(q_positions), float(rope_base), ctypes.byref(k.c()), ctypes.byref(v.c()),
+        _dev(PiK, "PiK"), _dev(PiV, "PiV"), pi_stride, _dev(S, "S"), _dev(cK, "cK"), _dev(cV, "cV"),
+        float(scale), _dev(out, "out"), _dtype_code(out), _ptr(scores_out), _ptr(d_status), _stream(stream)))
 
 
 def tq_dequantize(lay: Layout, is_key: bool, planes: Planes, n_vectors: int, Pi: torch.Tensor,

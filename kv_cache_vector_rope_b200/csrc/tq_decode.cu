@@ -23,6 +23,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
@@ -558,4 +559,78 @@ extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q,
   }
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_decode_attention launch: %s", cudaGetErrorString(e));
   return TQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// tq_decode_attention_noalloc: the same attention with the split-KV scratch in
+// a fixed device array owned by this library, for callers that cannot
+// allocate device memory when they call.
+//
+// The array lives in this file (64 MiB per device that loads the library, held
+// until the process exits). Host code must not hand the array's symbol to a
+// kernel: the symbol names a host-side stand-in. The device address is fetched
+// with cudaGetSymbolAddress once per device, with that device current, on the
+// first call made on it (that first call should therefore happen before any
+// stream capture). Every call shares the array and leaves its contents behind;
+// the kernels overwrite everything they read, so nothing needs clearing, but
+// calls that overlap on the GPU (different streams, or another host thread)
+// race on it.
+// ---------------------------------------------------------------------------
+static constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+namespace tq {
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+tq_status static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(TQ_ERR_UNSUPPORTED, "device index %d above %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(TQ_ERR_CUDA, "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+extern "C" tq_status tq_decode_attention_noalloc(const tq_layout* layout, const void* q, tq_dtype q_dtype,
+                                                 int32_t batch, int32_t hq, int32_t hkv, int32_t nq, int64_t n_ctx,
+                                                 int64_t ctx_stride, const int32_t* q_positions, float rope_base,
+                                                 const tq_planes* k, const tq_planes* v, const float* PiK,
+                                                 const float* PiV, int64_t pi_stride, const float* S, const float* cK,
+                                                 const float* cV, float scale, void* out, tq_dtype out_dtype,
+                                                 float* scores_out, int32_t* d_status, void* stream) {
+  using namespace tq;
+  clear_error();
+  const size_t need = tq_decode_workspace_bytes(layout, batch, hq, hkv, nq, n_ctx);
+  if (need == 0) {
+    // Let the regular entry point report exactly what is wrong with the arguments.
+    return tq_decode_attention(layout, q, q_dtype, batch, hq, hkv, nq, n_ctx, ctx_stride, q_positions, rope_base, k,
+                               v, PiK, PiV, pi_stride, S, cK, cV, scale, out, out_dtype, scores_out, nullptr, 0,
+                               d_status, stream);
+  }
+  if (need > kStaticScratchBytes)
+    return fail(TQ_ERR_UNSUPPORTED,
+                "tq_decode_attention_noalloc: this shape needs %zu bytes of scratch, above the fixed %zu-byte array; "
+                "use tq_decode_attention with a caller workspace",
+                need, kStaticScratchBytes);
+  void* scratch = nullptr;
+  tq_status st = static_scratch(&scratch);
+  if (st != TQ_OK) return st;
+  return tq_decode_attention(layout, q, q_dtype, batch, hq, hkv, nq, n_ctx, ctx_stride, q_positions, rope_base, k, v,
+                             PiK, PiV, pi_stride, S, cK, cV, scale, out, out_dtype, scores_out, scratch,
+                             kStaticScratchBytes, d_status, stream);
 }
