@@ -27,6 +27,7 @@
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
+#include "tq_decode_tc.h"
 
 namespace tq {
 namespace {
@@ -36,17 +37,6 @@ using namespace dev;
 constexpr int kT = 128;              // tokens per tile = threads of the main kernel
 constexpr int kTargetCtas = 1024;    // split heuristic target (shape-only, device independent)
 constexpr int kMaxRows = 8;          // query rows per main-kernel CTA
-
-struct DecodeShape {
-  int d, kbits, vbits;
-  int batch, hq, hkv, nq;
-  int64_t n_ctx, ctx_stride;
-  int rows_per_cta;   // R
-  int row_blocks;     // (hq/hkv*nq) / R
-  int n_splits;
-  int64_t chunk;      // tokens per split (multiple of kT)
-  int64_t n_rows;     // batch*hq*nq
-};
 
 int pick_rows(int group_rows) {
   for (int r = kMaxRows; r >= 1; r >>= 1)
@@ -84,33 +74,6 @@ size_t shape_workspace_bytes(const DecodeShape& s) {
   const size_t part = size_t(s.n_rows) * s.n_splits * (s.d + 2) * sizeof(float);
   return ((qs + 255) / 256) * 256 + part;
 }
-
-struct DecodeArgs {
-  DecodeShape sh;
-  const void* q;
-  int q_dtype;
-  const int32_t* q_pos;
-  double rope_base;
-  const uint8_t* kidx;
-  const uint32_t* ksign;
-  const float* knorm;
-  const float* krnorm;
-  const uint8_t* vidx;
-  const float* vnorm;
-  const float* PiK;
-  const float* PiV;
-  int64_t pi_stride;
-  const float* S;
-  const float* cK;
-  const float* cV;
-  float scale;
-  void* out;
-  int out_dtype;
-  float* scores_out;
-  float* qs;     // [n_rows][2][d]  q_rot then s
-  float* part;   // [n_rows][n_splits][d + 2]  acc..., m, l
-  int32_t* d_status;
-};
 
 // Query row index -> (b, h, n).
 __device__ __forceinline__ void row_coords(const DecodeShape& s, int64_t row, int& b, int& h, int& n) {
@@ -546,11 +509,19 @@ extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q,
   decode_prologue<<<static_cast<unsigned>(sh.n_rows), 128, (d * sizeof(double) + d * sizeof(float)), s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) {
+    // Tensor-core kernel where it applies (TQ_DECODE_PATH=v1|v2 selects a
+    // CUDA-core kernel instead; all compute the same attention).
+    const char* path = std::getenv("TQ_DECODE_PATH");
+    const bool cuda_core = path && (std::strcmp(path, "v1") == 0 || std::strcmp(path, "v2") == 0);
+    if (!cuda_core && tc_decode_supported(a)) {
+      e = tc_decode_launch(a, s);
+    } else {
     switch (d) {
       case 64: e = launch_main_rows<64>(a, s); break;
       case 128: e = launch_main_rows<128>(a, s); break;
       case 200: e = launch_main_rows<200>(a, s); break;
       default: return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: d=%d not built (64, 128, 200)", d);
+    }
     }
   }
   if (e == cudaSuccess) {
