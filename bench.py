@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--layers", type=int, default=32, help="layers of the cache (32 = the full workload)")
+    p.add_argument("--context", type=int, default=32768,
+                   help="context length (32768 = the full workload; smaller values only for profiling captures)")
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
@@ -210,7 +212,7 @@ def cpu_baseline(shape: synth.LlamaDecodeShape, budget_s: float, seed: int = 0) 
 def run_ours(args, world, rank):
     import kv_cache_vector_rope_b200 as tq
     dev = torch.device("cuda", torch.cuda.current_device())
-    shape = synth.LlamaDecodeShape()
+    shape = synth.LlamaDecodeShape(n_ctx=args.context)
     L = args.layers
     B, HQ, HKV, D, N = shape.batch, shape.hq, shape.hkv, shape.d, shape.n_ctx
     n_vec = B * HKV * N
