@@ -84,47 +84,123 @@ __device__ __forceinline__ void row_coords(const DecodeShape& s, int64_t row, in
 }
 
 // ---------------------------------------------------------------------------
-// 1. Prologue: q_rot = Pi_K[kv] RoPE(q), s = S q_rot (one CTA per query row).
+// Row blocks of the prologue and the combine: up to 16 query rows that share
+// one rotation (all rows when Pi is shared, else the G*nq rows of one
+// (batch, KV head) stream). Each CTA stages the d x d matrix once in shared
+// memory (row pitch d+1: conflict-free reads along either index) and applies
+// it to its rows; thread (i, group) owns coordinate i of RPG rows.
 // ---------------------------------------------------------------------------
-__global__ void decode_prologue(DecodeArgs a) {
-  extern __shared__ double pro_smem[];
+constexpr int kBlkRows = 16;
+constexpr int kBlkThreads = 256;
+
+struct RowBlocks {
+  int rows_per_group, blocks_per_group, n_blocks;
+};
+
+RowBlocks row_blocks(const DecodeShape& s, int64_t pi_stride) {
+  RowBlocks r{};
+  r.rows_per_group = pi_stride == 0 ? static_cast<int>(s.n_rows) : (s.hq / s.hkv) * s.nq;
+  r.blocks_per_group = (r.rows_per_group + kBlkRows - 1) / kBlkRows;
+  r.n_blocks = static_cast<int>(s.n_rows / r.rows_per_group) * r.blocks_per_group;
+  return r;
+}
+
+// Row groups per CTA: floor(256 / d) capped at 4, a power of two.
+inline int row_groups(int d) { return d <= 64 ? 4 : (d <= 128 ? 2 : 1); }
+inline size_t blk_smem_bytes(int d) { return sizeof(float) * (size_t(d) * (d + 1) + 2 * size_t(d) * kBlkRows); }
+
+// Stages the d x d row-major matrix M into Ms (pitch d+1): warp w copies rows
+// w, w+8, ...; lane l reads columns l, l+32, ... (coalesced).
+__device__ __forceinline__ void stage_matrix(float* Ms, const float* __restrict__ M, int d) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < d; i += kBlkThreads / 32)
+    for (int j = lane; j < d; j += 32) Ms[i * (d + 1) + j] = __ldg(M + int64_t(i) * d + j);
+}
+
+// out[r][i] = sum_j Ms[i][j] xs[j][r] (TRANS = false) or sum_j Ms[j][i] xs[j][r]
+// (TRANS = true) for the RPG rows of this thread's group; xs is j-major
+// [d][16]. Returns false for threads without a coordinate.
+template <int RPG, bool TRANS>
+__device__ __forceinline__ bool blk_matvec(const float* Ms, const float* xs, int d, float (&acc)[RPG], int& i, int& r0) {
+  const int t = threadIdx.x;
+  const int groups = kBlkRows / RPG;
+  if (t >= groups * d) return false;
+  i = t % d;
+  r0 = (t / d) * RPG;
+#pragma unroll
+  for (int u = 0; u < RPG; ++u) acc[u] = 0.f;
+  const int pitch = d + 1;
+  for (int j = 0; j < d; ++j) {
+    const float m = TRANS ? Ms[j * pitch + i] : Ms[i * pitch + j];
+    const float4* x4 = reinterpret_cast<const float4*>(xs + j * kBlkRows + r0);
+#pragma unroll
+    for (int u4 = 0; u4 < RPG / 4; ++u4) {
+      const float4 x = x4[u4];
+      acc[4 * u4 + 0] = fmaf(m, x.x, acc[4 * u4 + 0]);
+      acc[4 * u4 + 1] = fmaf(m, x.y, acc[4 * u4 + 1]);
+      acc[4 * u4 + 2] = fmaf(m, x.z, acc[4 * u4 + 2]);
+      acc[4 * u4 + 3] = fmaf(m, x.w, acc[4 * u4 + 3]);
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// 1. Prologue: q_rot = Pi_K[kv] RoPE(q), s = S q_rot for every query row.
+// ---------------------------------------------------------------------------
+template <int RPG>
+__global__ void __launch_bounds__(kBlkThreads) decode_prologue(DecodeArgs a, RowBlocks rb) {
+  extern __shared__ __align__(16) float blk_smem[];
   const DecodeShape& s = a.sh;
   const int d = s.d;
-  double* qd = pro_smem;            // [d] RoPE'd query
-  float* qr = reinterpret_cast<float*>(pro_smem + d);  // [d] q_rot
-  const int64_t row = blockIdx.x;
-  int b, h, n;
-  row_coords(s, row, b, h, n);
-  const int kv = h / (s.hq / s.hkv);
+  float* Ms = blk_smem;                       // [d][d+1]
+  float* xs = Ms + d * (d + 1);               // [d][16] RoPE'd queries
+  float* ys = xs + d * kBlkRows;              // [d][16] q_rot
+  const int g = blockIdx.x / rb.blocks_per_group, sub = blockIdx.x % rb.blocks_per_group;
+  const int64_t row0 = int64_t(g) * rb.rows_per_group + sub * kBlkRows;
+  const int cnt = min(kBlkRows, rb.rows_per_group - sub * kBlkRows);
+  const int kv = a.pi_stride ? g % s.hkv : 0;
+  stage_matrix(Ms, a.PiK + kv * a.pi_stride, d);
   const bool rope = a.q_pos != nullptr && a.rope_base > 0.0;
-  const int pos = rope ? a.q_pos[int64_t(b) * s.nq + n] : 0;
-  if (rope && pos < 0 && threadIdx.x == 0 && a.d_status) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
-  const int64_t qbase = row * d;
-  for (int i = threadIdx.x; i < d / 2; i += blockDim.x) {
-    double x0 = load_elem(a.q, a.q_dtype, qbase + i), x1 = load_elem(a.q, a.q_dtype, qbase + i + d / 2);
-    if (rope) {
-      double sn, cs;
-      sincos(rope_angle(pos, i, d, a.rope_base), &sn, &cs);
-      const double r0 = x0 * cs - x1 * sn, r1 = x0 * sn + x1 * cs;
-      x0 = r0;
-      x1 = r1;
+  for (int e = threadIdx.x; e < kBlkRows * (d / 2); e += kBlkThreads) {
+    const int r = e / (d / 2), i = e % (d / 2);
+    float x0 = 0.f, x1 = 0.f;
+    if (r < cnt) {
+      const int64_t row = row0 + r;
+      x0 = load_elem(a.q, a.q_dtype, row * d + i);
+      x1 = load_elem(a.q, a.q_dtype, row * d + i + d / 2);
+      if (rope) {
+        int b, h, n;
+        row_coords(s, row, b, h, n);
+        const int pos = a.q_pos[int64_t(b) * s.nq + n];
+        if (pos < 0 && a.d_status) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
+        double sn, cs;
+        sincos(rope_angle(pos, i, d, a.rope_base), &sn, &cs);
+        const double r0 = double(x0) * cs - double(x1) * sn, r1 = double(x0) * sn + double(x1) * cs;
+        x0 = static_cast<float>(r0);
+        x1 = static_cast<float>(r1);
+      }
     }
-    qd[i] = x0;
-    qd[i + d / 2] = x1;
+    xs[i * kBlkRows + r] = x0;
+    xs[(i + d / 2) * kBlkRows + r] = x1;
   }
   __syncthreads();
-  const float* Pi = a.PiK + kv * a.pi_stride;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    double acc = 0.0;
-    for (int j = 0; j < d; ++j) acc = fma(static_cast<double>(__ldg(Pi + int64_t(i) * d + j)), qd[j], acc);
-    qr[i] = static_cast<float>(acc);
-    a.qs[row * 2 * d + i] = static_cast<float>(acc);
+  float acc[RPG];
+  int i, r0;
+  if (blk_matvec<RPG, false>(Ms, xs, d, acc, i, r0)) {
+#pragma unroll
+    for (int u = 0; u < RPG; ++u) {
+      ys[i * kBlkRows + r0 + u] = acc[u];
+      if (r0 + u < cnt) a.qs[(row0 + r0 + u) * 2 * d + i] = acc[u];
+    }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    double acc = 0.0;
-    for (int j = 0; j < d; ++j) acc = fma(static_cast<double>(__ldg(a.S + int64_t(i) * d + j)), double(qr[j]), acc);
-    a.qs[row * 2 * d + d + i] = static_cast<float>(acc);
+  stage_matrix(Ms, a.S, d);
+  __syncthreads();
+  if (blk_matvec<RPG, false>(Ms, ys, d, acc, i, r0)) {
+#pragma unroll
+    for (int u = 0; u < RPG; ++u)
+      if (r0 + u < cnt) a.qs[(row0 + r0 + u) * 2 * d + d + i] = acc[u];
   }
 }
 
@@ -335,43 +411,85 @@ __global__ void __launch_bounds__(kT) decode_main(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// 3. Combine the splits and turn back by Pi_V^T (one CTA per query row).
+// 3. Combine the splits and turn back by Pi_V^T (a block of query rows per CTA).
 // ---------------------------------------------------------------------------
-__global__ void decode_combine(DecodeArgs a) {
-  extern __shared__ float cmb[];
+template <int RPG>
+__global__ void __launch_bounds__(kBlkThreads) decode_combine(DecodeArgs a, RowBlocks rb) {
+  extern __shared__ __align__(16) float blk_smem[];
   const DecodeShape& s = a.sh;
-  const int d = s.d;
-  const int64_t row = blockIdx.x;
-  int b, h, n;
-  row_coords(s, row, b, h, n);
-  const int kv = h / (s.hq / s.hkv);
-  const float* part = a.part + row * s.n_splits * (d + 2);
-  float M = -INFINITY;
-  for (int k = 0; k < s.n_splits; ++k) M = fmaxf(M, part[k * (d + 2) + d]);
-  float L = 0.f;
-  for (int k = 0; k < s.n_splits; ++k) {
-    const float mk = part[k * (d + 2) + d];
-    if (mk > -INFINITY) L += expf(mk - M) * part[k * (d + 2) + d + 1];
-  }
-  float* o = cmb;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float acc = 0.f;
-    for (int k = 0; k < s.n_splits; ++k) {
-      const float mk = part[k * (d + 2) + d];
-      if (mk > -INFINITY) acc += expf(mk - M) * part[k * (d + 2) + i];
+  const int d = s.d, ns = s.n_splits;
+  float* Ms = blk_smem;                       // [d][d+1] Pi_V
+  float* os = Ms + d * (d + 1);               // [d][16] merged rotated outputs
+  float* wl = os + d * kBlkRows;              // [16] 1 / L per row; [16] max per row
+  const int g = blockIdx.x / rb.blocks_per_group, sub = blockIdx.x % rb.blocks_per_group;
+  const int64_t row0 = int64_t(g) * rb.rows_per_group + sub * kBlkRows;
+  const int cnt = min(kBlkRows, rb.rows_per_group - sub * kBlkRows);
+  const int kv = a.pi_stride ? g % s.hkv : 0;
+  stage_matrix(Ms, a.PiV + kv * a.pi_stride, d);
+  // Row maxima and softmax denominators: warp w handles rows w and w + 8.
+  {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < kBlkRows; r += kBlkThreads / 32) {
+      float M = -INFINITY, L = 0.f;
+      if (r < cnt) {
+        const float* part = a.part + (row0 + r) * ns * (d + 2);
+        for (int k = lane; k < ns; k += 32) M = fmaxf(M, part[k * (d + 2) + d]);
+        M = warp_max(M);
+        for (int k = lane; k < ns; k += 32) {
+          const float mk = part[k * (d + 2) + d];
+          if (mk > -INFINITY) L += __expf(mk - M) * part[k * (d + 2) + d + 1];
+        }
+        L = warp_sum(L);
+      }
+      if (lane == 0) {
+        wl[r] = (r < cnt && L > 0.f) ? 1.f / L : 0.f;
+        wl[kBlkRows + r] = M;
+      }
     }
-    o[i] = acc / L;
   }
   __syncthreads();
-  const float* Pi = a.PiV + kv * a.pi_stride;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < d; ++i) acc = fmaf(__ldg(Pi + int64_t(i) * d + j), o[i], acc);
-    if (a.out_dtype == 0)
-      reinterpret_cast<float*>(a.out)[row * d + j] = acc;
-    else
-      reinterpret_cast<__nv_bfloat16*>(a.out)[row * d + j] = __float2bfloat16(acc);
+  // Merged rotated output o[r][i] = sum_k e^(m_k - M) acc_k[i] / L.
+  for (int e = threadIdx.x; e < kBlkRows * d; e += kBlkThreads) {
+    const int r = e / d, i = e % d;
+    float o = 0.f;
+    if (r < cnt) {
+      const float* part = a.part + (row0 + r) * ns * (d + 2);
+      const float M = wl[kBlkRows + r];
+      for (int k = 0; k < ns; ++k) {
+        const float mk = part[k * (d + 2) + d];
+        if (mk > -INFINITY) o = fmaf(__expf(mk - M), part[k * (d + 2) + i], o);
+      }
+      o *= wl[r];
+    }
+    os[i * kBlkRows + r] = o;
   }
+  __syncthreads();
+  float acc[RPG];
+  int j, r0;
+  if (blk_matvec<RPG, true>(Ms, os, d, acc, j, r0)) {
+#pragma unroll
+    for (int u = 0; u < RPG; ++u) {
+      if (r0 + u >= cnt) continue;
+      const int64_t row = row0 + r0 + u;
+      if (a.out_dtype == 0)
+        reinterpret_cast<float*>(a.out)[row * d + j] = acc[u];
+      else
+        reinterpret_cast<__nv_bfloat16*>(a.out)[row * d + j] = __float2bfloat16(acc[u]);
+    }
+  }
+}
+
+template <bool COMBINE>
+cudaError_t launch_blk(const DecodeArgs& a, cudaStream_t st) {
+  const RowBlocks rb = row_blocks(a.sh, a.pi_stride);
+  const size_t smem = blk_smem_bytes(a.sh.d) + (COMBINE ? 2 * kBlkRows * sizeof(float) : 0);
+  const int rg = row_groups(a.sh.d);
+  auto kern = COMBINE ? (rg == 4 ? decode_combine<4> : rg == 2 ? decode_combine<8> : decode_combine<16>)
+                      : (rg == 4 ? decode_prologue<4> : rg == 2 ? decode_prologue<8> : decode_prologue<16>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<static_cast<unsigned>(rb.n_blocks), kBlkThreads, smem, st>>>(a, rb);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -506,8 +624,7 @@ extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q,
                                     ((size_t(sh.n_rows) * 2 * d * sizeof(float) + 255) / 256) * 256);
   a.d_status = d_status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  decode_prologue<<<static_cast<unsigned>(sh.n_rows), 128, (d * sizeof(double) + d * sizeof(float)), s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_blk<false>(a, s);
   if (e == cudaSuccess) {
     // Tensor-core kernel where it applies (TQ_DECODE_PATH=v1|v2 selects a
     // CUDA-core kernel instead; all compute the same attention).
@@ -525,8 +642,7 @@ extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q,
     }
   }
   if (e == cudaSuccess) {
-    decode_combine<<<static_cast<unsigned>(sh.n_rows), 128, d * sizeof(float), s>>>(a);
-    e = cudaGetLastError();
+    e = launch_blk<true>(a, s);
   }
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_decode_attention launch: %s", cudaGetErrorString(e));
   return TQ_OK;

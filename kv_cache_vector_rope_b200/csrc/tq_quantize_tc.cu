@@ -7,32 +7,35 @@
 // index per coordinate of y/||x||) and Etapa 2 (sign of S times the residual,
 // residual norm); gist.science "TurboESM ..." section 2A (RoPE before Pi).
 //
-// Per CTA (persistent, one per SM), tiles of 128 vectors:
-//   warp 0      TMA: 128 x d bf16 tile -> shared memory (128-byte swizzle)
-//   warp 1      MMA issuer (one thread) + TMEM owner:
-//                 Y = X (Pi1 + Pi2 + Pi3)^T        3 chains, A/B in smem
-//                 P = (R1 + R2) (S1 + S2)^T         R1S1 + R1S2 + R2S1, A in TMEM
-//               Pi = Pi1+Pi2+Pi3 and S = S1+S2 are bf16 splits made in the
-//               prologue; x is bf16, so X Pi_t^T is exact per product and only
-//               the fp32 accumulation rounds.
-//   warps 2-9   epilogue, two warpgroups splitting the d columns: norms from
-//               the smem tile, codes by binary search on ||x|| t_j, residual r
-//               (fp32 kept in TMEM, bf16 splits R1/R2 for the second MMA), sign
-//               bits, packing and stores.
-// TMEM: Y/P double buffer (2d columns), R1|R2 (d), r fp32 (d).
+// Per CTA (persistent, one per SM), tiles of 128 vectors; tile i of a CTA
+// uses TMEM slot i % 2 and is finished by epilogue warpgroup i % 2, so the two
+// warpgroups work on alternate tiles and never wait for each other:
+//   warp 0      TMA: 128 x d bf16 tile -> shared memory (128-byte swizzle),
+//               2-4 stage ring; a stage is released by the MMA that read it
+//   warp 1      TMEM owner and single-thread MMA issuer:
+//                 Y = X (Pi3 + Pi2 + Pi1)^T      bf16 splits, small parts first
+//                 P = (R1 + R2) (S1 + S2)^T      fp16 splits, A from TMEM
+//                                                (R2 S1 + R1 S2 + R1 S1)
+//   warps 2-5   epilogue warpgroup 0, warps 6-9 epilogue warpgroup 1; thread =
+//               vector (TMEM lane). Per tile: ||y|| from the accumulator, codes
+//               by binary search against ||y|| t_j, residual r, fp16 splits of
+//               r 2^k (k from ||y||, so r 2^k stays below 2^14) into TMEM for P,
+//               sign bits from P, packing and stores.
+// TMEM slot (keys): Y/P accumulator (d columns) | R1 (d/2) | R2 (d/2).
 //
-// Exactness. A code is decided in fp32 only when y is farther than
-// 3e-6 ||x|| from every boundary it was compared with; otherwise that
-// coordinate's y is recomputed in fp64 from x and Pi (warp-cooperative) and
-// the code decided there. A sign is decided from the MMA only when
-// |p| > 1e-4 ||r||; otherwise p is recomputed in fp64 from the fp32 residual,
-// and if that value is within 1e-5 ||r|| of zero, from a residual rebuilt
-// entirely in fp64 (every coordinate of the row, one lane per coordinate).
+// Exactness. The norm is ||y|| = ||Pi x|| in fp32 (Pi orthogonal; error
+// ~1e-7 relative). A code is decided in fp32 only when y is farther than
+// 3e-7 ||y|| from every boundary it was compared with, a sign only when |p|
+// exceeds 1.5e-5 ||r||. A row with any other coordinate or sign is flagged
+// (sign bit of its stored ||r|| for keys, of ||x|| for values) and a second
+// launch, quantize_fixup, recomputes every flagged row exactly in fp64 (one
+// warp per row: ||x||, y = Pi x, codes, r, p = S r) and overwrites it.
 //
 // Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT in *d_status and
 // the CTA drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -49,13 +52,19 @@ using namespace sm100;
 using dev::warp_sum;
 
 constexpr int kThreads = 320;         // 10 warps
-// Guard bands. The fp32 accumulation of the 3-way split rotation errs by
-// ~1e-7 ||x|| per coordinate (std), the 2x2-way split projection by ~3e-6 ||r||,
-// and the fp32 residual moves an fp64 projection by ~5e-7 ||r||: each band is
-// more than 20 standard deviations of the error it covers.
-constexpr float kCodeGuard = 3e-6f;
-constexpr float kSignGuard = 1e-4f;
-constexpr double kSignGuard2 = 1e-5;
+// Guard bands, set from the measured errors of this formulation on B200: the
+// rotation accumulator errs by at most 7.4e-8 ||x|| per coordinate (typically
+// 2e-8), and the projection of the fp32 residual by at most 2.5e-6 ||r||
+// (the residual inherits the rotation's error). Each band is 4-6x the
+// largest error seen over ~5e5 samples.
+constexpr float kCodeGuard = 3e-7f;
+constexpr float kSignGuard = 1.5e-5f;
+
+constexpr int pow2_at_least(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
 
 template <int D, bool KEY>
 struct Cfg {
@@ -63,29 +72,25 @@ struct Cfg {
   static constexpr int kKSteps = D / 16;
   static constexpr int kTileBytes = kM * D * 2;
   static constexpr int kMatBytes = D * D * 2;
-  static constexpr int kStages = (KEY && D == 128) ? 1 : (D == 128 ? 3 : 4);
+  static constexpr int kStages = (D == 128) ? (KEY ? 2 : 3) : 4;
   static constexpr int kSSplits = KEY ? 2 : 0;
-  static constexpr int kColY = 0;                    // buffers at 0 and D
-  static constexpr int kColR1 = 2 * D;
-  static constexpr int kColR2 = 2 * D + D / 2;
-  static constexpr int kColR32 = 3 * D;
-  static constexpr int kTmemCols = KEY ? 4 * D : 2 * D;
+  static constexpr int kSlotCols = KEY ? 2 * D : D;  // accumulator | R1 | R2
+  static constexpr int kColR1 = D;
+  static constexpr int kColR2 = D + D / 2;
+  static constexpr int kTmemCols = pow2_at_least(2 * kSlotCols);
   static constexpr int kChunks = D / 32;             // 32-column chunks
-  static constexpr int kChunksPerWg = kChunks / 2;
   // Shared memory plan (offsets from a 1024-aligned base).
   static constexpr int kOffPi = 0;
   static constexpr int kOffS = kOffPi + 3 * kMatBytes;
   static constexpr int kOffX = kOffS + kSSplits * kMatBytes;
   static constexpr int kOffBar = kOffX + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 2 + 1;
+  // full[st], empty[st], yfull[2], rfull[2], pfull[2], accfree[2], drain
+  static constexpr int kNumBars = 2 * kStages + 8 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  // misc: tmem base (4) + abort (4) + cent[16] + bnd[16] + nrm partials [2][128] double + rsq [2][128] float
+  // misc: tmem base (4) + abort (4) + r-scale exponent shift (4) + pad (4) + cent[16] + bnd[16]
   static constexpr int kOffCent = kOffMisc + 16;
   static constexpr int kOffBnd = kOffCent + 64;
-  static constexpr int kOffNrm = kOffBnd + 64;
-  static constexpr int kOffRsq = kOffNrm + 2 * 2 * kM * 8;     // norm partials double-buffered by tile parity
-  static constexpr int kOffScratch = kOffRsq + 2 * kM * 4;   // 8 warps x 32 floats
-  static constexpr int kSmemBytes = kOffScratch + 8 * 32 * 4 + 1024;   // + alignment slack
+  static constexpr int kSmemBytes = kOffBnd + 64 + 1024;   // + alignment slack
 };
 
 struct TcArgs {
@@ -103,22 +108,7 @@ struct TcArgs {
   int32_t* d_status;
 };
 
-// Barrier over the 256 epilogue threads that also ORs a predicate across them,
-// so every epilogue warp takes the same abort decision.
-__device__ __forceinline__ bool epi_sync_or(bool p) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "barrier.cta.red.or.pred po, 1, 256, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(p))
-      : "memory");
-  return r != 0;
-}
-
-// Splits v into bf16 terms hi (+ mid (+ lo)) that add up to v to ~2^-25.
+// Splits v into bf16 terms hi + mid + lo that add up to v to ~2^-25.
 __device__ __forceinline__ void split3(float v, __nv_bfloat16& a, __nv_bfloat16& b, __nv_bfloat16& c) {
   a = __float2bfloat16_rn(v);
   const float r1 = v - __bfloat162float(a);
@@ -126,15 +116,50 @@ __device__ __forceinline__ void split3(float v, __nv_bfloat16& a, __nv_bfloat16&
   c = __float2bfloat16_rn(r1 - __bfloat162float(b));
 }
 
-// Exact (fp64) y_i = Pi_i . x_row, warp-cooperative (all lanes call it).
+// x[4 lane .. 4 lane + KPL) of a bf16 row (KPL = D/32 elements per lane) in fp64.
 template <int D>
-__device__ __noinline__ double exact_y(const float* __restrict__ M, int i, const __nv_bfloat16* __restrict__ xrow) {
+__device__ __forceinline__ void lane_x(const __nv_bfloat16* __restrict__ xrow, double (&xk)[D / 32]) {
   const int lane = threadIdx.x & 31;
-  double acc = 0.0;
+  if constexpr (D == 128) {
+    const uint2 v = *reinterpret_cast<const uint2*>(xrow + 4 * lane);
+    xk[0] = __uint_as_float(v.x << 16);
+    xk[1] = __uint_as_float(v.x & 0xffff0000u);
+    xk[2] = __uint_as_float(v.y << 16);
+    xk[3] = __uint_as_float(v.y & 0xffff0000u);
+  } else {
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(xrow + 2 * lane);
+    xk[0] = __uint_as_float(v << 16);
+    xk[1] = __uint_as_float(v & 0xffff0000u);
+  }
+}
+
+// Row i of Pi times the lane's slice of x, in fp64 (no reduction).
+template <int D>
+__device__ __forceinline__ double lane_dot(const float* __restrict__ Pi, int i, const double (&xk)[D / 32]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (D == 128) {
+    const float4 w = __ldg(reinterpret_cast<const float4*>(Pi + i * D) + lane);
+    return fma(double(w.x), xk[0], fma(double(w.y), xk[1], fma(double(w.z), xk[2], double(w.w) * xk[3])));
+  } else {
+    const float2 w = __ldg(reinterpret_cast<const float2*>(Pi + i * D) + lane);
+    return fma(double(w.x), xk[0], double(w.y) * xk[1]);
+  }
+}
+
+// Sum over lanes of v[m] for every m, returned in lane m (31 exchanges).
+__device__ __forceinline__ double transpose_reduce32(double (&v)[32]) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int j = lane; j < D; j += 32)
-    acc = fma(static_cast<double>(__ldg(M + i * D + j)), static_cast<double>(__bfloat162float(xrow[j])), acc);
-  return warp_sum(acc);
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool up = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const double send = up ? v[i] : v[i + s];
+      const double keep = up ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
 }
 
 // Exact code of y64 (zero vector: u = 0).
@@ -149,63 +174,41 @@ __device__ __forceinline__ int exact_code(double y64, double nrm64, const float*
   return c;
 }
 
-// p_i = S_i . r for the row held by lane L, with r the fp32 residual stored in
-// TMEM columns [col_r, col_r + D) of each lane (warp-cooperative).
-template <int D>
-__device__ __noinline__ double p_from_tmem(const float* __restrict__ S, int i, int L, uint32_t lane_addr, uint32_t col_r) {
-  const int lane = threadIdx.x & 31;
-  double sv[D / 32];
+// Code of y against thresholds th[] (strict: ties go to the lower code) and
+// the distance from y to the nearest boundary of its cell.
+template <int BITS>
+__device__ __forceinline__ int code_of(float y, const float (&th)[(1 << BITS) - 1], float& dmin) {
+  if (BITS == 3) {
+    const bool b2 = y > th[3];
+    const float tA = b2 ? th[5] : th[1];
+    const bool b1 = y > tA;
+    const float tB = b2 ? (b1 ? th[6] : th[4]) : (b1 ? th[2] : th[0]);
+    const bool b0 = y > tB;
+    dmin = fminf(fabsf(y - th[3]), fminf(fabsf(y - tA), fabsf(y - tB)));
+    return (b2 ? 4 : 0) | (b1 ? 2 : 0) | (b0 ? 1 : 0);
+  } else if (BITS == 2) {
+    const bool b1 = y > th[1];
+    const float tA = b1 ? th[2] : th[0];
+    const bool b0 = y > tA;
+    dmin = fminf(fabsf(y - th[1]), fabsf(y - tA));
+    return (b1 ? 2 : 0) | (b0 ? 1 : 0);
+  } else {
+    int c = 0;
+    dmin = INFINITY;
 #pragma unroll
-  for (int c4 = 0; c4 < D / 32; ++c4) sv[c4] = static_cast<double>(__ldg(S + i * D + c4 * 32 + lane));
-  double acc = 0.0;
-#pragma unroll
-  for (int c4 = 0; c4 < D / 32; ++c4) {
-    uint32_t rr[32];
-    tmem_ld32(lane_addr + col_r + c4 * 32, rr);
-    tmem_ld_wait();
-    float mine = 0.f;
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const float vL = __shfl_sync(0xffffffffu, __uint_as_float(rr[u]), L);
-      if (lane == u) mine = vL;
+    for (int j = 0; j < (1 << BITS) - 1; ++j) {
+      c += (y > th[j]) ? 1 : 0;
+      dmin = fminf(dmin, fabsf(y - th[j]));
     }
-    acc = fma(sv[c4], static_cast<double>(mine), acc);
+    return c;
   }
-  return warp_sum(acc);
-}
-
-// p_i with the residual of row xrow rebuilt in fp64: lane j' owns the
-// coordinates j = j' + 32 m, computing y_j, its code and r_j exactly.
-template <int D, int NB>
-__device__ __noinline__ double p_rebuild(const float* __restrict__ Pi, const float* __restrict__ S, int i,
-                                         const __nv_bfloat16* __restrict__ xrow, double nrm64, const float* bnd,
-                                         const float* cent) {
-  const int lane = threadIdx.x & 31;
-  double acc = 0.0;
-#pragma unroll 1
-  for (int m = 0; m < D / 32; ++m) {
-    const int j = lane + 32 * m;
-    double y = 0.0;
-    const float4* row = reinterpret_cast<const float4*>(Pi + j * D);
-#pragma unroll 4
-    for (int k4 = 0; k4 < D / 4; ++k4) {
-      const float4 w = __ldg(row + k4);
-      y = fma(static_cast<double>(w.x), static_cast<double>(__bfloat162float(xrow[4 * k4 + 0])), y);
-      y = fma(static_cast<double>(w.y), static_cast<double>(__bfloat162float(xrow[4 * k4 + 1])), y);
-      y = fma(static_cast<double>(w.z), static_cast<double>(__bfloat162float(xrow[4 * k4 + 2])), y);
-      y = fma(static_cast<double>(w.w), static_cast<double>(__bfloat162float(xrow[4 * k4 + 3])), y);
-    }
-    const int c = exact_code<NB>(y, nrm64, bnd);
-    const double r = y - nrm64 * static_cast<double>(cent[c]);
-    acc = fma(static_cast<double>(__ldg(S + i * D + j)), r, acc);
-  }
-  return warp_sum(acc);
 }
 
 template <int D, bool KEY, int BITS>
 __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
   using C = Cfg<D, KEY>;
   constexpr int kNb = (1 << BITS) - 1;
+  constexpr int kRowBytes = D * BITS / 8;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* pi_s = sm + C::kOffPi;
@@ -214,35 +217,44 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::kStages;
-  uint64_t* yfull = bars + 2 * C::kStages;          // [2]
-  uint64_t* accfree = yfull + 2;                      // [2]
-  uint64_t* rfull = accfree + 2;                      // [1]
-  uint64_t* pfull = rfull + 1;                        // [2]
-  uint64_t* drain = pfull + 2;                        // [1] final MMA drain
+  uint64_t* yfull = bars + 2 * C::kStages;           // [2]
+  uint64_t* rfull = yfull + 2;                        // [2]
+  uint64_t* pfull = rfull + 2;                        // [2]
+  uint64_t* accfree = pfull + 2;                      // [2]
+  uint64_t* drain = accfree + 2;                      // [1] final MMA drain
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
+  int* rshift_s = reinterpret_cast<int*>(sm + C::kOffMisc + 8);
   float* cent_s = reinterpret_cast<float*>(sm + C::kOffCent);
   float* bnd_s = reinterpret_cast<float*>(sm + C::kOffBnd);
-  double* nrm_part = reinterpret_cast<double*>(sm + C::kOffNrm);
-  float* rsq_part = reinterpret_cast<float*>(sm + C::kOffRsq);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (a.n + C::kM - 1) / C::kM;
+  const int my_tiles = (n_tiles > blockIdx.x) ? static_cast<int>((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
 
   // ---------------------------------------------------------------- prologue
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 8);
+      mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&yfull[b], 1);
-      mbar_init(&accfree[b], 8);
+      mbar_init(&rfull[b], 4);
       mbar_init(&pfull[b], 1);
+      mbar_init(&accfree[b], 4);
     }
-    mbar_init(rfull, 8);
     mbar_init(drain, 1);
     *abort_s = 0;
+    // r 2^k must stay below 2^14 for fp16: |r| <= (1 + max|c|) ||y||.
+    float lim = 1.f;
+    for (int k = 0; k <= kNb; ++k) lim = fmaxf(lim, 1.f + fabsf(a.cent[k]));
+    int sh = 0;
+    while (lim > 2.f && sh < 60) {
+      lim *= 0.5f;
+      ++sh;
+    }
+    *rshift_s = sh;
     mbar_fence_init();
   }
   if (tid < 16) cent_s[tid] = tid <= kNb ? a.cent[tid] : 0.f;
@@ -251,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     tmem_alloc(tmem_base_s, C::kTmemCols);
     tmem_relinquish();
   }
-  // bf16 splits of Pi (3) and S (2) in the K-major 128B-swizzled layout.
+  // bf16 splits of Pi (3) and fp16 splits of S (2), K-major, 128B-swizzled.
   for (int e = tid; e < D * D; e += kThreads) {
     const int i = e / D, j = e % D;
     const uint32_t off = sw128_offset(i, j, D);
@@ -261,9 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     *reinterpret_cast<__nv_bfloat16*>(pi_s + C::kMatBytes + off) = m;
     *reinterpret_cast<__nv_bfloat16*>(pi_s + 2 * C::kMatBytes + off) = l;
     if (KEY) {
-      split3(__ldg(a.S + e), h, m, l);
-      *reinterpret_cast<__nv_bfloat16*>(s_s + off) = h;
-      *reinterpret_cast<__nv_bfloat16*>(s_s + C::kMatBytes + off) = m;
+      const float sv = __ldg(a.S + e);
+      const __half sh = __float2half_rn(sv);
+      const __half sl = __float2half_rn(sv - __half2float(sh));
+      *reinterpret_cast<__half*>(s_s + off) = sh;
+      *reinterpret_cast<__half*>(s_s + C::kMatBytes + off) = sl;
     }
   }
   fence_proxy_async_smem();
@@ -284,10 +298,10 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   if (warp == 0) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      int it = 0;
-      int armed[C::kStages > 0 ? C::kStages : 1];
+      int armed[C::kStages];
       for (int s = 0; s < C::kStages; ++s) armed[s] = 0;
-      for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+      for (int it = 0; it < my_tiles; ++it) {
+        const int64_t t = blockIdx.x + int64_t(it) * gridDim.x;
         const int st = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
         if (*abort_s) break;
@@ -306,49 +320,48 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_bf16_f32(128, D);
-      const uint32_t pi_base = smem_u32(pi_s), s_base = smem_u32(s_s), x_base = smem_u32(x_s);
-      // Descriptors differ only in the start-address field (low 14 bits,
-      // address >> 4): build the bases once, add constant offsets per K-step.
-      const uint64_t pi_desc0 = desc_k_sw128(pi_base), s_desc0 = desc_k_sw128(s_base), x_desc0 = desc_k_sw128(x_base);
+      constexpr uint32_t kIdescY = idesc_bf16_f32(128, D);
+      constexpr uint32_t kIdescP = (1u << 4) | (static_cast<uint32_t>(D >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+      const uint64_t pi_desc0 = desc_k_sw128(smem_u32(pi_s)), s_desc0 = desc_k_sw128(smem_u32(s_s)),
+                     x_desc0 = desc_k_sw128(smem_u32(x_s));
       auto issue_y = [&](int it) {
         const int st = it % C::kStages;
         const int b = it & 1;
-        const uint32_t d_tmem = tmem + C::kColY + b * D;
+        const uint32_t d_tmem = tmem + b * C::kSlotCols;
         const uint64_t xa = x_desc0 + static_cast<uint64_t>((st * C::kTileBytes) >> 4);
+        // Small split first: the fp32 accumulator then rounds at the scale of
+        // the large terms only during the last K-steps.
 #pragma unroll
-        for (int sp = 0; sp < 3; ++sp) {
+        for (int q = 0; q < 3; ++q) {
+          const int sp = 2 - q;
 #pragma unroll
           for (int k = 0; k < C::kKSteps; ++k) {
             constexpr int kAtomA = 128 * 128, kAtomB = D * 128;
             const uint64_t ad = xa + static_cast<uint64_t>(((k >> 2) * kAtomA + (k & 3) * 32) >> 4);
             const uint64_t bd = pi_desc0 + static_cast<uint64_t>((sp * C::kMatBytes + (k >> 2) * kAtomB + (k & 3) * 32) >> 4);
-            umma_ss(d_tmem, ad, bd, kIdesc, (sp | k) != 0);
+            umma_ss(d_tmem, ad, bd, kIdescY, (q | k) != 0);
           }
         }
         umma_commit(&yfull[b]);
+        umma_commit(&empty[st]);        // the X stage is free once Y is computed
       };
       auto issue_p = [&](int it) {
         const int b = it & 1;
-        const uint32_t d_tmem = tmem + C::kColY + b * D;
-        // (A, B) pairs: R1 S1, R1 S2, R2 S1.
+        const uint32_t slot = tmem + b * C::kSlotCols;
+        // (A, B) pairs, small terms first: R2 S1, R1 S2, R1 S1.
 #pragma unroll
         for (int pr = 0; pr < 3; ++pr) {
-          const uint32_t acol = (pr == 2) ? C::kColR2 : C::kColR1;
+          const uint32_t acol = (pr == 0) ? C::kColR2 : C::kColR1;
           const int boff = (pr == 1) ? C::kMatBytes : 0;
 #pragma unroll
           for (int k = 0; k < C::kKSteps; ++k) {
             constexpr int kAtomB = D * 128;
             const uint64_t bd = s_desc0 + static_cast<uint64_t>((boff + (k >> 2) * kAtomB + (k & 3) * 32) >> 4);
-            umma_ts(d_tmem, tmem + acol + k * 8, bd, kIdesc, (pr | k) != 0);
+            umma_ts(slot, slot + acol + k * 8, bd, kIdescP, (pr | k) != 0);   // kind::f16, f16 A/B per kIdescP
           }
         }
         umma_commit(&pfull[b]);
       };
-      // Issue whatever is ready: Y of the next tile (its X landed and its
-      // accumulator buffer is free) and, for keys, P of the oldest tile whose
-      // residual is in TMEM. Neither waits behind the other.
-      const int my_tiles = (n_tiles > blockIdx.x) ? static_cast<int>((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
       int ny = 0, np = 0;
       uint64_t last = globaltimer_ns();
       while (KEY ? (np < my_tiles) : (ny < my_tiles)) {
@@ -365,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
             progress = true;
           }
         }
-        if (KEY && np < ny && mbar_try_wait(rfull, np & 1)) {
+        if (KEY && np < ny && mbar_try_wait(&rfull[np & 1], (np >> 1) & 1)) {
           tc_fence_after();
           issue_p(np);
           ++np;
@@ -381,204 +394,167 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     }
   } else {
     // --------------------------------------------------------------- epilogue
-    const int ew = warp - 2;                 // 0..7
-    const int g = ew >> 2;                   // column half
+    const int wg = (warp - 2) >> 2;          // 0 or 1: tiles it with it % 2 == wg
     const int q = warp & 3;                  // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;           // row within the tile
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    float th[kNb > 0 ? kNb : 1];
-    int it = 0;
-    for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-      const int st = it % C::kStages;
-      const uint32_t ph = (it / C::kStages) & 1;
-      const int b = it & 1;
-      const uint32_t bph = (it >> 1) & 1;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16) + wg * C::kSlotCols;
+    const int rshift = *rshift_s;
+    float th[kNb];
+    for (int it = wg; it < my_tiles; it += 2) {
+      const int64_t t = blockIdx.x + int64_t(it) * gridDim.x;
+      const uint32_t ph = (it >> 1) & 1;
       const int64_t v = t * C::kM + row;
       const bool valid = v < a.n;
-      // ||x||^2 from the shared tile (this warpgroup's half of x).
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], ph));
-      {
-        const unsigned char* xt = x_s + st * C::kTileBytes;
-        double ss = 0.0;
-#pragma unroll
-        for (int cc = 0; cc < D / 16; ++cc) {
-          const int k0 = g * (D / 2) + cc * 8;
-          const uint4 w = *reinterpret_cast<const uint4*>(xt + sw128_offset(row, k0, C::kM));
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float lo = __uint_as_float(ws[h] << 16), hi = __uint_as_float(ws[h] & 0xffff0000u);
-            ss += static_cast<double>(lo * lo) + static_cast<double>(hi * hi);
-          }
-        }
-        nrm_part[((it & 1) * 2 + g) * C::kM + row] = ss;
+      if (!__all_sync(0xffffffffu, mbar_wait(&yfull[wg], ph))) {
+        if (lane == 0) fail();
+        break;
       }
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&yfull[b], bph));
       tc_fence_after();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);     // X tile no longer needed
-      if (!ok && lane == 0) fail();
-      if (epi_sync_or(!ok || *abort_s != 0)) break;
-      const double nrm64 = sqrt(nrm_part[(it & 1) * 2 * C::kM + row] + nrm_part[((it & 1) * 2 + 1) * C::kM + row]);
-      const float nrm = static_cast<float>(nrm64);
+      // Pass 1: ||y||^2 from the accumulator.
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < C::kChunks; ++ch) {
+        uint32_t yb[32];
+        tmem_ld32(lane_addr + ch * 32, yb);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+          const float y0 = __uint_as_float(yb[k]), y1 = __uint_as_float(yb[k + 1]);
+          const float y2 = __uint_as_float(yb[k + 2]), y3 = __uint_as_float(yb[k + 3]);
+          s0 = fmaf(y0, y0, s0);
+          s1 = fmaf(y1, y1, s1);
+          s2 = fmaf(y2, y2, s2);
+          s3 = fmaf(y3, y3, s3);
+        }
+      }
+      const float nrm = sqrtf((s0 + s1) + (s2 + s3));
       const float band = kCodeGuard * nrm;
 #pragma unroll
-      for (int j = 0; j < kNb; ++j) th[j] = nrm * bnd_s[j];
-
-      uint32_t codew[C::kChunksPerWg][BITS];
+      for (int j = 0; j < kNb; ++j) th[j] = nrm > 0.f ? nrm * bnd_s[j] : bnd_s[j];
+      // fp16 scale of r: 2^(13 - e - rshift) with nrm = m 2^e, m in [0.5, 1).
+      float rscale = 1.f;
+      if (KEY) {
+        const int ex = static_cast<int>((__float_as_uint(nrm) >> 23) & 0xFFu);
+        if (ex != 0) {
+          int be = 266 - ex - rshift;
+          be = be < 1 ? 1 : (be > 254 ? 254 : be);
+          rscale = __uint_as_float(static_cast<uint32_t>(be) << 23);
+        }
+      }
+      uint32_t rowflag = 0;                  // any coordinate or sign near its decision
+      uint32_t codew[C::kChunks][BITS];
       float rsq = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < C::kChunksPerWg; ++cc) {
-        const int ch = g * C::kChunksPerWg + cc;
-        uint32_t ybits[32];
-        tmem_ld32(lane_addr + C::kColY + b * D + ch * 32, ybits);
+      for (int ch = 0; ch < C::kChunks; ++ch) {
+        uint32_t yb[32];
+        tmem_ld32(lane_addr + ch * 32, yb);
         tmem_ld_wait();
         int code[32];
         float r[32];
         uint32_t flags = 0;
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float y = __uint_as_float(ybits[k]);
-          int c;
+          const float y = __uint_as_float(yb[k]);
           float dmin;
-          if (BITS == 3) {
-            const bool b2 = y > th[3];
-            const float tA = b2 ? th[5] : th[1];
-            const bool b1 = y > tA;
-            const float tB = b2 ? (b1 ? th[6] : th[4]) : (b1 ? th[2] : th[0]);
-            const bool b0 = y > tB;
-            c = (b2 ? 4 : 0) + (b1 ? 2 : 0) + (b0 ? 1 : 0);
-            dmin = fminf(fabsf(y - th[3]), fminf(fabsf(y - tA), fabsf(y - tB)));
-          } else {
-            c = 0;
-            dmin = INFINITY;
-#pragma unroll
-            for (int j = 0; j < kNb; ++j) {
-              c += (y > th[j]) ? 1 : 0;
-              dmin = fminf(dmin, fabsf(y - th[j]));
-            }
-          }
-          if (dmin <= band) flags |= 1u << k;
+          const int c = code_of<BITS>(y, th, dmin);
+          if (dmin < band) flags |= 1u << k;
           code[k] = c;
           r[k] = fmaf(-nrm, cent_s[c], y);
         }
-        if (!valid) flags = 0;
-        // Exact fp64 decision for every coordinate near a boundary: one
-        // (lane, coordinate) at a time, the whole warp computing its dot product.
-#pragma unroll 1
-        for (unsigned m = __ballot_sync(0xffffffffu, flags != 0u); m != 0u;
-             m = __ballot_sync(0xffffffffu, flags != 0u)) {
-          const int L = __ffs(m) - 1;
-          const int kL = __ffs(__shfl_sync(0xffffffffu, flags, L)) - 1;
-          const int64_t vL = __shfl_sync(0xffffffffu, v, L);
-          const double y64 = exact_y<D>(a.Pi, ch * 32 + kL, a.x + vL * a.row_stride);
-          if (lane == L) {
-            const int c = exact_code<kNb>(y64, nrm64, bnd_s);
-            const float rr = static_cast<float>(y64 - nrm64 * static_cast<double>(cent_s[c]));
-            flags &= ~(1u << kL);
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              if (k == kL) {
-                code[k] = c;
-                r[k] = rr;
-              }
-          }
-        }
+        rowflag |= flags;
         // Pack this chunk's codes (32 codes -> BITS words).
 #pragma unroll
-        for (int w = 0; w < BITS; ++w) codew[cc][w] = 0u;
+        for (int w = 0; w < BITS; ++w) codew[ch][w] = 0u;
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           const int bp = k * BITS;
-          codew[cc][bp >> 5] |= static_cast<uint32_t>(code[k]) << (bp & 31);
-          if ((bp & 31) + BITS > 32) codew[cc][(bp >> 5) + 1] |= static_cast<uint32_t>(code[k]) >> (32 - (bp & 31));
+          codew[ch][bp >> 5] |= static_cast<uint32_t>(code[k]) << (bp & 31);
+          if ((bp & 31) + BITS > 32) codew[ch][(bp >> 5) + 1] |= static_cast<uint32_t>(code[k]) >> (32 - (bp & 31));
         }
         if (KEY) {
-          uint32_t r1[16], r2[16], rb[32];
+          uint32_t r1[16], r2[16];
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
             rsq = fmaf(r[k], r[k], fmaf(r[k + 1], r[k + 1], rsq));
-            const __nv_bfloat162 h = __floats2bfloat162_rn(r[k], r[k + 1]);
-            const float2 hf = __bfloat1622float2(h);
-            const __nv_bfloat162 l = __floats2bfloat162_rn(r[k] - hf.x, r[k + 1] - hf.y);
+            const float a0 = r[k] * rscale, a1 = r[k + 1] * rscale;
+            const __half2 h = __floats2half2_rn(a0, a1);
+            const float2 hf = __half22float2(h);
+            const __half2 l = __floats2half2_rn(a0 - hf.x, a1 - hf.y);
             r1[k / 2] = *reinterpret_cast<const uint32_t*>(&h);
             r2[k / 2] = *reinterpret_cast<const uint32_t*>(&l);
-            rb[k] = __float_as_uint(r[k]);
-            rb[k + 1] = __float_as_uint(r[k + 1]);
           }
           tmem_st16(lane_addr + C::kColR1 + ch * 16, r1);
           tmem_st16(lane_addr + C::kColR2 + ch * 16, r2);
-          tmem_st32(lane_addr + C::kColR32 + ch * 32, rb);
         }
       }
-      // Stores of this warpgroup's part of the row.
-      if (valid) {
-        constexpr int kRowBytes = D * BITS / 8;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(a.idx + v * kRowBytes) + g * C::kChunksPerWg * BITS;
-#pragma unroll
-        for (int cc = 0; cc < C::kChunksPerWg; ++cc)
-#pragma unroll
-          for (int w = 0; w < BITS; ++w) dst[cc * BITS + w] = codew[cc][w];
-        if (g == 0) a.norm[v] = nrm;
-      }
-      if (!KEY) {
+      if (KEY) {
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&accfree[b]);
-        continue;
+        if (lane == 0) mbar_arrive(&rfull[wg]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      rsq_part[g * C::kM + row] = rsq;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(rfull);
-      if (epi_sync_or(*abort_s != 0)) break;
-      const float rn = sqrtf(rsq_part[row] + rsq_part[C::kM + row]);
-      // On a timeout the loop ends at the next iteration's barrier; results of
-      // this tile are then meaningless and *d_status says so.
-      if (!__all_sync(0xffffffffu, mbar_wait(&pfull[b], bph)) && lane == 0) fail();
-      tc_fence_after();
-      const float sband = kSignGuard * rn;
+      // Stores of the row's codes and norm (overlap the projection MMA).
+      if (valid) {
+        uint32_t flat[kRowBytes / 4];
 #pragma unroll
-      for (int cc = 0; cc < C::kChunksPerWg; ++cc) {
-        const int ch = g * C::kChunksPerWg + cc;
-        uint32_t pbits[32];
-        tmem_ld32(lane_addr + C::kColY + b * D + ch * 32, pbits);
-        tmem_ld_wait();
-        uint32_t word = 0, flags = 0;
+        for (int ch = 0; ch < C::kChunks; ++ch)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p = __uint_as_float(pbits[k]);
-          word |= (p >= 0.f ? 1u : 0u) << k;
-          if (fabsf(p) <= sband) flags |= 1u << k;
+          for (int w = 0; w < BITS; ++w) flat[ch * BITS + w] = codew[ch][w];
+        uint8_t* dst = a.idx + v * kRowBytes;
+        if constexpr (kRowBytes % 16 == 0) {
+#pragma unroll
+          for (int u = 0; u < kRowBytes / 16; ++u)
+            reinterpret_cast<uint4*>(dst)[u] = make_uint4(flat[4 * u], flat[4 * u + 1], flat[4 * u + 2], flat[4 * u + 3]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < kRowBytes / 8; ++u) reinterpret_cast<uint2*>(dst)[u] = make_uint2(flat[2 * u], flat[2 * u + 1]);
         }
-        if (!valid) flags = 0;
-        // fp64 recomputation of p_i = S_i . r for signs near zero.
-#pragma unroll 1
-        for (unsigned m = __ballot_sync(0xffffffffu, flags != 0u); m != 0u;
-             m = __ballot_sync(0xffffffffu, flags != 0u)) {
-          const int L = __ffs(m) - 1;
-          const int kL = __ffs(__shfl_sync(0xffffffffu, flags, L)) - 1;
-          const int i = ch * 32 + kL;
-          const double p1 = p_from_tmem<D>(a.S, i, L, lane_addr, C::kColR32);
-          const float rnL = __shfl_sync(0xffffffffu, rn, L);
-          bool bit = p1 >= 0.0;
-          if (fabs(p1) <= kSignGuard2 * rnL) {
-            const int64_t vL = __shfl_sync(0xffffffffu, v, L);
-            const double nL = __shfl_sync(0xffffffffu, nrm64, L);
-            bit = p_rebuild<D, kNb>(a.Pi, a.S, i, a.x + vL * a.row_stride, nL, bnd_s, cent_s) >= 0.0;
-          }
-          if (lane == L) {
-            word = bit ? (word | (1u << kL)) : (word & ~(1u << kL));
-            flags &= ~(1u << kL);
-          }
-        }
-        if (valid) a.sign[v * C::kChunks + ch] = word;
+        // Values: a row with an undecided code is flagged by the sign bit of
+        // its norm (keys carry the flag on ||r||); quantize_fixup redoes it.
+        a.norm[v] = (!KEY && rowflag) ? -nrm : nrm;
       }
-      if (valid && g == 0) a.rnorm[v] = rn;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accfree[b]);
+      if (KEY) {
+        const float rn = sqrtf(rsq);
+        const float sband = kSignGuard * rn * rscale;
+        if (!__all_sync(0xffffffffu, mbar_wait(&pfull[wg], ph))) {
+          if (lane == 0) fail();
+          break;
+        }
+        tc_fence_after();
+        uint32_t words[C::kChunks];
+#pragma unroll
+        for (int ch = 0; ch < C::kChunks; ++ch) {
+          uint32_t pbits[32];
+          tmem_ld32(lane_addr + ch * 32, pbits);
+          tmem_ld_wait();
+          uint32_t word = 0, flags = 0;
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float p = __uint_as_float(pbits[k]);
+            word |= (p >= 0.f ? 1u : 0u) << k;
+            if (fabsf(p) < sband) flags |= 1u << k;
+          }
+          rowflag |= flags;
+          words[ch] = word;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accfree[wg]);
+        if (valid) {
+          uint32_t* sdst = a.sign + v * C::kChunks;
+          if constexpr (C::kChunks == 4) {
+            reinterpret_cast<uint4*>(sdst)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < C::kChunks; ++ch) sdst[ch] = words[ch];
+          }
+          a.rnorm[v] = rowflag ? __uint_as_float(__float_as_uint(rn) | 0x80000000u) : rn;
+        }
+      } else {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accfree[wg]);
+      }
     }
   }
 
@@ -595,6 +571,89 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     }
     __syncwarp();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Exact recomputation of flagged rows (fp64, one warp per row). The flag is the
+// sign bit of the row's stored ||r|| (keys) or ||x|| (values); every output of
+// the row is rewritten, the flag cleared.
+// ---------------------------------------------------------------------------
+template <int D, bool KEY, int BITS>
+__device__ __noinline__ void fix_row(const TcArgs& a, int64_t v, const float* cent, const float* bnd) {
+  constexpr int kNb = (1 << BITS) - 1;
+  constexpr int G = D / 32;
+  const int lane = threadIdx.x & 31;
+  double xk[G];
+  lane_x<D>(a.x + v * a.row_stride, xk);
+  double nn = 0.0;
+#pragma unroll
+  for (int u = 0; u < G; ++u) nn = fma(xk[u], xk[u], nn);
+  const double n64 = sqrt(warp_sum(nn));
+  // y_j, code_j and r_j for j = 32 g + lane.
+  double r[G];
+  uint32_t* idx = reinterpret_cast<uint32_t*>(a.idx + v * (D * BITS / 8));
+#pragma unroll 1
+  for (int g = 0; g < G; ++g) {
+    double part[32];
+#pragma unroll
+    for (int m = 0; m < 32; ++m) part[m] = lane_dot<D>(a.Pi, 32 * g + m, xk);
+    const double y = transpose_reduce32(part);
+    const uint32_t c = static_cast<uint32_t>(exact_code<kNb>(y, n64, bnd));
+    r[g] = y - n64 * static_cast<double>(cent[c]);
+    // Codes of this group -> BITS packed words (little-endian bit stream).
+    const int o = BITS * lane;
+#pragma unroll
+    for (int w = 0; w < BITS; ++w) {
+      uint32_t val = 0u;
+      if ((o >> 5) == w) val |= c << (o & 31);
+      if ((o >> 5) == w - 1 && (o & 31) + BITS > 32) val |= c >> (32 - (o & 31));
+      const uint32_t word = __reduce_or_sync(0xffffffffu, val);
+      if (lane == 0) idx[g * BITS + w] = word;
+    }
+  }
+  if (lane == 0) a.norm[v] = static_cast<float>(n64);
+  if (KEY) {
+    double rr = 0.0;
+#pragma unroll
+    for (int g = 0; g < G; ++g) rr = fma(r[g], r[g], rr);
+    const double rn = sqrt(warp_sum(rr));
+#pragma unroll 1
+    for (int h = 0; h < G; ++h) {
+      double part[32];
+#pragma unroll
+      for (int m = 0; m < 32; ++m) {
+        double acc = 0.0;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          acc = fma(static_cast<double>(__ldg(a.S + (32 * h + m) * D + 32 * g + lane)), r[g], acc);
+        part[m] = acc;
+      }
+      const double p = transpose_reduce32(part);          // lane m: p_(32 h + m)
+      const uint32_t word = __ballot_sync(0xffffffffu, p >= 0.0);
+      if (lane == 0) a.sign[v * G + h] = word;
+    }
+    if (lane == 0) a.rnorm[v] = static_cast<float>(rn);
+  }
+}
+
+template <int D, bool KEY, int BITS>
+__global__ void __launch_bounds__(256) quantize_fixup(TcArgs a) {
+  __shared__ float cent_s[16], bnd_s[16];
+  if (threadIdx.x < 16) {
+    cent_s[threadIdx.x] = threadIdx.x <= (1 << BITS) - 1 ? a.cent[threadIdx.x] : 0.f;
+    bnd_s[threadIdx.x] = threadIdx.x < (1 << BITS) - 1 ? a.bnd[threadIdx.x] : 0.f;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_id = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const float* flagp = KEY ? a.rnorm : a.norm;
+  for (int64_t base = warp_id * 32; base < a.n; base += n_warps * 32) {
+    const int64_t row = base + lane;
+    const bool f = row < a.n && (__float_as_uint(flagp[row]) >> 31) != 0u;
+    for (unsigned m = __ballot_sync(0xffffffffu, f); m != 0u; m &= m - 1u)
+      fix_row<D, KEY, BITS>(a, base + (__ffs(m) - 1), cent_s, bnd_s);
   }
 }
 
@@ -629,6 +688,10 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& map, cudaStream_t st) 
   const int64_t tiles = (a.n + 127) / 128;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   quantize_tc_kernel<D, KEY, BITS><<<grid, kThreads, C::kSmemBytes, st>>>(map, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t fix_ctas = (a.n + 255) / 256;
+  quantize_fixup<D, KEY, BITS><<<static_cast<int>(fix_ctas < 4 * sms ? fix_ctas : 4 * sms), 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
