@@ -577,10 +577,16 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 // Exact recomputation of flagged rows (fp64, one warp per row). The flag is the
 // sign bit of the row's stored ||r|| (keys) or ||x|| (values); every output of
-// the row is rewritten, the flag cleared.
+// the row is rewritten and the flag cleared. One CTA per SM scans a contiguous
+// range of rows into a shared-memory list; if the list is not empty it stages
+// Pi (and S) in shared memory and its warps take list entries one at a time.
 // ---------------------------------------------------------------------------
+constexpr int kFixThreads = 1024;
+constexpr int kFixList = 16384;      // rows scanned per round (list capacity)
+
 template <int D, bool KEY, int BITS>
-__device__ __noinline__ void fix_row(const TcArgs& a, int64_t v, const float* cent, const float* bnd) {
+__device__ __noinline__ void fix_row(const TcArgs& a, int64_t v, const float* Pis, const float* Ss, const float* cent,
+                                     const float* bnd) {
   constexpr int kNb = (1 << BITS) - 1;
   constexpr int G = D / 32;
   const int lane = threadIdx.x & 31;
@@ -597,7 +603,13 @@ __device__ __noinline__ void fix_row(const TcArgs& a, int64_t v, const float* ce
   for (int g = 0; g < G; ++g) {
     double part[32];
 #pragma unroll
-    for (int m = 0; m < 32; ++m) part[m] = lane_dot<D>(a.Pi, 32 * g + m, xk);
+    for (int m = 0; m < 32; ++m) {
+      const float* row = Pis + (32 * g + m) * D + G * lane;
+      double acc = 0.0;
+#pragma unroll
+      for (int u = 0; u < G; ++u) acc = fma(static_cast<double>(row[u]), xk[u], acc);
+      part[m] = acc;
+    }
     const double y = transpose_reduce32(part);
     const uint32_t c = static_cast<uint32_t>(exact_code<kNb>(y, n64, bnd));
     r[g] = y - n64 * static_cast<double>(cent[c]);
@@ -625,8 +637,7 @@ __device__ __noinline__ void fix_row(const TcArgs& a, int64_t v, const float* ce
       for (int m = 0; m < 32; ++m) {
         double acc = 0.0;
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-          acc = fma(static_cast<double>(__ldg(a.S + (32 * h + m) * D + 32 * g + lane)), r[g], acc);
+        for (int g = 0; g < G; ++g) acc = fma(static_cast<double>(Ss[(32 * h + m) * D + 32 * g + lane]), r[g], acc);
         part[m] = acc;
       }
       const double p = transpose_reduce32(part);          // lane m: p_(32 h + m)
@@ -637,23 +648,57 @@ __device__ __noinline__ void fix_row(const TcArgs& a, int64_t v, const float* ce
   }
 }
 
+template <int D, bool KEY>
+constexpr size_t fix_smem_bytes() {
+  return sizeof(float) * size_t(D) * D * (KEY ? 2 : 1) + sizeof(int) * kFixList;
+}
+
 template <int D, bool KEY, int BITS>
-__global__ void __launch_bounds__(256) quantize_fixup(TcArgs a) {
+__global__ void __launch_bounds__(kFixThreads, 1) quantize_fixup(TcArgs a) {
+  extern __shared__ __align__(16) float fix_smem[];
+  float* Pis = fix_smem;                               // [D][D]
+  float* Ss = Pis + D * D;                             // [D][D] (keys)
+  int* list = reinterpret_cast<int*>(Ss + (KEY ? D * D : 0));
   __shared__ float cent_s[16], bnd_s[16];
+  __shared__ int cnt, taken;
   if (threadIdx.x < 16) {
     cent_s[threadIdx.x] = threadIdx.x <= (1 << BITS) - 1 ? a.cent[threadIdx.x] : 0.f;
     bnd_s[threadIdx.x] = threadIdx.x < (1 << BITS) - 1 ? a.bnd[threadIdx.x] : 0.f;
   }
-  __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int64_t warp_id = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const float* flagp = KEY ? a.rnorm : a.norm;
-  for (int64_t base = warp_id * 32; base < a.n; base += n_warps * 32) {
-    const int64_t row = base + lane;
-    const bool f = row < a.n && (__float_as_uint(flagp[row]) >> 31) != 0u;
-    for (unsigned m = __ballot_sync(0xffffffffu, f); m != 0u; m &= m - 1u)
-      fix_row<D, KEY, BITS>(a, base + (__ffs(m) - 1), cent_s, bnd_s);
+  const int64_t per = (a.n + gridDim.x - 1) / gridDim.x;
+  const int64_t r0 = int64_t(blockIdx.x) * per;
+  const int64_t r1 = r0 + per < a.n ? r0 + per : a.n;
+  bool staged = false;
+  for (int64_t w0 = r0; w0 < r1; w0 += kFixList) {
+    const int64_t w1 = w0 + kFixList < r1 ? w0 + kFixList : r1;
+    if (threadIdx.x == 0) {
+      cnt = 0;
+      taken = 0;
+    }
+    __syncthreads();
+    for (int64_t row = w0 + threadIdx.x; row < w1; row += blockDim.x)
+      if (__float_as_uint(flagp[row]) >> 31) list[atomicAdd(&cnt, 1)] = static_cast<int>(row - w0);
+    __syncthreads();
+    const int total = cnt;
+    if (total == 0) continue;
+    if (!staged) {
+      for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) {
+        reinterpret_cast<float4*>(Pis)[e] = __ldg(reinterpret_cast<const float4*>(a.Pi) + e);
+        if (KEY) reinterpret_cast<float4*>(Ss)[e] = __ldg(reinterpret_cast<const float4*>(a.S) + e);
+      }
+      __syncthreads();
+      staged = true;
+    }
+    for (;;) {
+      int e = 0;
+      if (lane == 0) e = atomicAdd(&taken, 1);
+      e = __shfl_sync(0xffffffffu, e, 0);
+      if (e >= total) break;
+      fix_row<D, KEY, BITS>(a, w0 + list[e], Pis, Ss, cent_s, bnd_s);
+    }
+    __syncthreads();
   }
 }
 
@@ -690,8 +735,13 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& map, cudaStream_t st) 
   quantize_tc_kernel<D, KEY, BITS><<<grid, kThreads, C::kSmemBytes, st>>>(map, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t fix_ctas = (a.n + 255) / 256;
-  quantize_fixup<D, KEY, BITS><<<static_cast<int>(fix_ctas < 4 * sms ? fix_ctas : 4 * sms), 256, 0, st>>>(a);
+  constexpr size_t fix_smem = fix_smem_bytes<D, KEY>();
+  e = cudaFuncSetAttribute(quantize_fixup<D, KEY, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(fix_smem));
+  if (e != cudaSuccess) return e;
+  const int64_t fix_ctas = (a.n + kFixList - 1) / kFixList;
+  quantize_fixup<D, KEY, BITS><<<static_cast<int>(fix_ctas < sms ? (fix_ctas < 1 ? 1 : fix_ctas) : sms), kFixThreads,
+                                 fix_smem, st>>>(a);
   return cudaGetLastError();
 }
 
