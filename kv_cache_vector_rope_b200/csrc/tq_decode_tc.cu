@@ -8,27 +8,35 @@
 //
 // Both contractions of decode run on the tensor cores over operands rebuilt
 // from the packed cache in on-chip memory, with exact integer arithmetic:
-//   scores  S[t][r] = sum_i c_K[code_ti] q_r,i  and  sum_i bit_ti s_r,i.
-//           A (TMEM, one lane per token): the key codebook value of every
-//           coordinate as three int8 limbs (c = sc (a1 + a2/128 + a3/128^2))
-//           and the sign bits as 0/1 bytes. B (smem): q_rot and s = S q_rot
-//           of the four rows as three int8 limbs each. int32 accumulation is
-//           exact. Three codebook limbs are needed because a codebook error
-//           repeats on every coordinate holding that code: with two limbs the
-//           2-bit codebook alone moves scores by ~1e-4 of |q||k|/d.
-//   values  O[i][r] = sum_t c_V[code_ti] w_r,t with w = p ||v||.
-//           A (smem, M-major): the value codebook value as two int8 limbs
-//           per coordinate, one 128-byte row per token. B (smem): the tile's
-//           weights as two int8 limbs per row with a per-tile scale. Each
-//           tile's int32 result is folded into fp32 accumulators (one
-//           coordinate per thread) with the online-softmax correction.
+//   scores  A (TMEM, one lane per token), 128 columns per tile:
+//             a1 | a2 | a3   the key codebook value of every coordinate as
+//                            three int8 limbs, c = sc (a1 + a2/128 + a3/128^2)
+//             sgn            the sign bits, masked in place: byte 16 j + b is
+//                            byte b of the sign row AND (1 << j), i.e. bit
+//                            8 b + j of the sketch times 2^j (unsigned)
+//           B (smem, K-major): per query row four int8 limbs of q_rot and of
+//           s' = s 2^-(i mod 8) (sign-chunk rows permuted to match). Limb
+//           products of equal weight 128^-w go to the same int32 column: the
+//           a1, a2, a3 chunks use B tiles whose limb columns are shifted by
+//           0, 1, 2, so D column 4 r + w holds sum_{l+m=w} a_l q_m.
+//   values  O[i][n] = sum_t c_V[code_ti] w_t,n: A (smem, M-major) the value
+//           codebook as two int8 limbs per coordinate, one 128-byte row per
+//           token; B the tile's weights w = p ||v|| / s_tile as two int8 limbs
+//           per query row, s_tile = max_t p ||v|| / 127 of that row, found as
+//           2^(max_t z_t - m log2 e) with z = score log2 e + log2 ||v||.
+// Online softmax: the running maximum per row only moves when a score of the
+// tile exceeds it (a vote over the softmax warps; the tile maximum is reduced
+// only then); the per-warp maxima of z are published before the same vote
+// barrier, so an ordinary tile costs one barrier. l is kept per thread and
+// summed once per work item; corrections and scales are uniform across the
+// softmax threads and stay in registers.
 // Roles (448 threads, one persistent CTA per SM):
-//   warp 0   bulk copies of the packed index / sign planes into a 3-stage ring
-//   warp 1   TMEM owner and single-thread tcgen05.mma issuer
-//   WG A     key dequantisation into TMEM          (thread = token)
-//   WG B     value dequantisation into smem        (thread = token)
-//   WG C     score epilogue, online softmax, weight limbs (thread = token)
-//            and the value epilogue                (thread = coordinate)
+//   warp 0     bulk copies of the packed index / sign planes into a 3-stage ring
+//   warp 1     TMEM owner and single-thread tcgen05.mma issuer
+//   warps 2-5  key operand generation into TMEM        (thread = token)
+//   warps 6-9  value operand generation into smem      (thread = token)
+//   warps 10-13 scores, softmax and weight limbs       (thread = token),
+//             the value epilogue                       (thread = coordinate)
 // Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT and the CTA
 // drains its copies and MMAs before it frees TMEM and returns.
 #include <cuda.h>
@@ -52,37 +60,33 @@ constexpr int kStages = 3;
 constexpr int kThreadsTc = 448;        // 14 warps
 constexpr int kRowsTc = 4;
 
-// TMEM columns (32-bit): A_score [0,128): a1 | a2 | a3 | sign bytes (32 each);
-// D_score x2 at 128, 192 (64 each: four 16-column chains); D_o x2 at 256, 288.
-constexpr uint32_t kColA = 0, kColDs = 128, kColDo = 256, kTmemColsTc = 512;
-constexpr uint32_t kDsCols = 64;
+// TMEM columns (32-bit): A_score x2 at 0, 128 (a1 | a2 | a3 | sgn, 32 each);
+// D_score x2 at 256, 288 (mse 16 | sgn 16); D_o x2 at 320, 352 (limb chains).
+constexpr uint32_t kColA = 0, kColDs = 256, kColDo = 320, kTmemColsTc = 512;
 
-// Instruction descriptor, kind::i8: s32 D, signed A/B, M = 128, N = 16.
-__host__ __device__ constexpr uint32_t idesc_i8(bool a_mn_major) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((16u >> 3) << 17) |
-         ((128u >> 4) << 24);
+// Instruction descriptor, kind::i8: s32 D, M = 128, N = 16.
+__host__ __device__ constexpr uint32_t idesc_i8(bool a_signed, bool a_mn_major) {
+  return (2u << 4) | ((a_signed ? 1u : 0u) << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((16u >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 template <int KB>
 struct TcSm {
   static constexpr int kRbk = kD * KB / 8;
   static constexpr int kStageBytes = kTT * (kRbk + 16 + 48);       // kidx | ksign | vidx
-  static constexpr int kOffStage = 0;
-  static constexpr int kOffVh = 3 * ((kStageBytes + 1023) / 1024) * 1024;   // 1024-aligned
+  static constexpr int kStageStride = ((kStageBytes + 1023) / 1024) * 1024;
+  static constexpr int kOffVh = kStages * kStageStride;            // 1024-aligned
   static constexpr int kVhBytes = 2 * kTT * 128;                    // two limbs x 128 tokens x 128 B
   static constexpr int kOffP = kOffVh + 2 * kVhBytes;               // 2 x [16 rows x 128 B]
-  static constexpr int kOffB = kOffP + 2 * 2048;                    // 2 items x (Q limbs | S limbs)
-  static constexpr int kOffBar = kOffB + 2 * 4096;
-  static constexpr int kNumBars = 2 * kStages + 2 + 2 * 2 * 6 + 2 + 1;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  // misc: tmem base, abort | item scales [2][16] | ring [2][8] | scratch [16] |
-  // reductions [4 warps][8] | codebook limb tables (ka1 ka2 ka3 va1 va2, 4 words each) | scales (key, value)
-  static constexpr int kOffScale = kOffMisc + 16;
-  static constexpr int kOffRing = kOffScale + 2 * 16 * 4;
-  static constexpr int kOffScr = kOffRing + 2 * 8 * 4;
-  static constexpr int kOffRed = kOffScr + 16 * 4;
-  static constexpr int kOffTab = kOffRed + 4 * 8 * 4;
-  static constexpr int kBytes = kOffTab + 32 * 4 + 1024;
+  static constexpr int kOffB = kOffP + 2 * 2048;                    // 2 items x (B1 | B2 | B3 | Bs)
+  static constexpr int kOffBar = kOffB + 2 * 4 * 2048;
+  static constexpr int kNumBars = 2 * kStages + 2 * 11 + 1;
+  static constexpr int kOffMisc = ((kOffBar + kNumBars * 8 + 15) / 16) * 16;
+  static constexpr int kOffZ = kOffMisc + 16;                       // [2 tiles][4 warps][4] max z
+  static constexpr int kOffRed = kOffZ + 2 * 4 * 4 * 4;             // [4 warps][16]
+  static constexpr int kOffRed2 = kOffRed + 4 * 16 * 4;             // [4 warps][4]
+  static constexpr int kOffTab = kOffRed2 + 4 * 4 * 4;              // ka1 ka2 ka3 va1 va2 (4 words) + 2 scales
+  static constexpr int kBytes = kOffTab + 22 * 4 + 1024;
 };
 
 struct TcDecodeArgs {
@@ -137,19 +141,18 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
   return d;
 }
 
-// 8 three-bit codes (24 bits) -> two PRMT selectors of four nibbles each.
-__device__ __forceinline__ void spread3(uint32_t x, uint32_t& lo, uint32_t& hi) {
-  const uint32_t y = (x & 0xFFFu) | ((x << 4) & 0x0FFF0000u);
-  const uint32_t z = (y & 0x00070007u) | ((y << 1) & 0x00700070u) | ((y << 2) & 0x07000700u) | ((y << 3) & 0x70007000u);
-  lo = z & 0xFFFFu;
-  hi = z >> 16;
+// 8 three-bit codes (bits 0..23 of x; bits above ignored) -> one word of
+// eight nibbles c0..c7; PRMT reads the low 16 bits as the selector of c0..c3.
+__device__ __forceinline__ uint32_t nibbles3(uint32_t x) {
+  const uint32_t y = (x & 0xFFFu) | ((x << 4) & 0x0FFF0000u);          // c0-3 | c4-7 in halves
+  const uint32_t z = (y & 0x003F003Fu) | ((y << 2) & 0x3F003F00u);     // two codes per byte
+  return (z & 0x07070707u) | ((z << 1) & 0x70707070u);                 // one code per nibble
 }
-// 8 two-bit codes (16 bits) -> nibble selectors.
-__device__ __forceinline__ void spread2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+// 8 two-bit codes (bits 0..15 of x) -> eight nibbles.
+__device__ __forceinline__ uint32_t nibbles2(uint32_t x) {
   const uint32_t y = (x & 0xFFu) | ((x << 8) & 0x00FF0000u);
-  const uint32_t z = (y & 0x00030003u) | ((y << 2) & 0x00300030u) | ((y << 4) & 0x03000300u) | ((y << 6) & 0x30003000u);
-  lo = z & 0xFFFFu;
-  hi = z >> 16;
+  const uint32_t z = (y & 0x000F000Fu) | ((y << 4) & 0x0F000F00u);
+  return (z & 0x03030303u) | ((z << 2) & 0x30303030u);
 }
 // Byte lookup of four codes in a 16-entry table given as four words (codes
 // 0-3 | 4-7 | 8-11 | 12-15); `nib` holds the four 4-bit codes.
@@ -163,21 +166,7 @@ __device__ __forceinline__ uint32_t lut16(const uint32_t (&t)[4], uint32_t nib) 
                         ((mk & 0xF000u) ? 0xFF000000u : 0u);
   return (lo & ~mask) | (hi & mask);
 }
-// Four sign bits -> four 0/1 bytes.
-__device__ __forceinline__ uint32_t bits4_to_bytes(uint32_t n4) { return (n4 * 0x00204081u) & 0x01010101u; }
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
-               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
@@ -202,13 +191,19 @@ __device__ __forceinline__ void umma_i8_ts(uint32_t d, uint32_t a, uint64_t b, u
 __device__ __forceinline__ uint32_t sw_byte(int r, int k) {
   return static_cast<uint32_t>(r * 128 + ((((k >> 4) ^ (r & 7))) << 4) + (k & 15));
 }
-// Three int8 limbs of x / scale (|x / scale| <= 127): x ~ scale (l0 + l1/128 + l2/16384).
-__device__ __forceinline__ void limbs3(float x, float inv_scale, int& l0, int& l1, int& l2) {
-  const float r0 = x * inv_scale;
-  l0 = __float2int_rn(r0);
-  const float r1 = (r0 - static_cast<float>(l0)) * 128.f;
-  l1 = __float2int_rn(r1);
-  l2 = __float2int_rn((r1 - static_cast<float>(l1)) * 128.f);
+// Four int8 limbs of x (|x| <= 127): x ~ l0 + l1/128 + l2/128^2 + l3/128^3.
+__device__ __forceinline__ void limbs4(float x, int (&l)[4]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    l[u] = __float2int_rn(x);
+    x = (x - static_cast<float>(l[u])) * 128.f;
+  }
+}
+__device__ __forceinline__ float limb_sum4(const uint32_t* d) {
+  float v = static_cast<float>(static_cast<int>(d[3]));
+  v = fmaf(v, 1.f / 128.f, static_cast<float>(static_cast<int>(d[2])));
+  v = fmaf(v, 1.f / 128.f, static_cast<float>(static_cast<int>(d[1])));
+  return fmaf(v, 1.f / 128.f, static_cast<float>(static_cast<int>(d[0])));
 }
 
 template <int KB>
@@ -221,9 +216,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Sm::kOffBar);
   uint64_t* st_full = bars;                       // [3]
   uint64_t* st_empty = bars + kStages;            // [3]
-  uint64_t* a_full = bars + 2 * kStages;          // [1]
-  uint64_t* a_free = a_full + 1;                  // [1]
-  uint64_t* s_full = a_free + 1;                  // [2]
+  uint64_t* a_full = bars + 2 * kStages;          // [2]
+  uint64_t* a_free = a_full + 2;                  // [2]
+  uint64_t* s_full = a_free + 2;                  // [2]
   uint64_t* ds_free = s_full + 2;                 // [2]
   uint64_t* vh_full = ds_free + 2;                // [2]
   uint64_t* vh_free = vh_full + 2;                // [2]
@@ -235,10 +230,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
   uint64_t* drain = b_full + 2;                   // [1]
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Sm::kOffMisc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + Sm::kOffMisc + 4);
-  float* item_scale = reinterpret_cast<float*>(sm + Sm::kOffScale);   // [2][16]: sq[4], ss[4], ssum[4]
-  float* ring = reinterpret_cast<float*>(sm + Sm::kOffRing);          // [2][8]: corr[4], sp[4]
-  float* red = reinterpret_cast<float*>(sm + Sm::kOffRed);            // [4 warps][8]
-  float* scr = reinterpret_cast<float*>(sm + Sm::kOffScr);            // [16]
+  float* zred = reinterpret_cast<float*>(sm + Sm::kOffZ);             // [2][4 warps][4]
+  float* red = reinterpret_cast<float*>(sm + Sm::kOffRed);            // [4 warps][16]
+  float* red2 = reinterpret_cast<float*>(sm + Sm::kOffRed2);          // [4 warps][4]
   uint32_t* tab = reinterpret_cast<uint32_t*>(sm + Sm::kOffTab);      // ka1 ka2 ka3 va1 va2 (4 words each)
   float* cb_scale = reinterpret_cast<float*>(sm + Sm::kOffTab + 20 * 4);   // key, value codebook scales
 
@@ -250,9 +244,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
       mbar_init(&st_full[s], 1);
       mbar_init(&st_empty[s], 8);
     }
-    mbar_init(a_full, 4);
-    mbar_init(a_free, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&a_full[b], 4);
+      mbar_init(&a_free[b], 1);
       mbar_init(&s_full[b], 1);
       mbar_init(&ds_free[b], 4);
       mbar_init(&vh_full[b], 4);
@@ -275,6 +269,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
     tmem_alloc(tmem_base_s, kTmemColsTc);
     tmem_relinquish();
   }
+  // Rows 8-15 of both weight tiles stay zero (only 2 limbs x 4 rows are used).
+  for (int e = tid; e < 2 * 1024 / 16; e += kThreadsTc) {
+    const int b = e / 64, o = e % 64;
+    reinterpret_cast<uint4*>(sm + Sm::kOffP + b * 2048 + 1024)[o] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
           const int nt = static_cast<int>((te - t0 < kTT) ? te - t0 : kTT);
           const uint32_t bk = nt * kRbk, bs = nt * 16, bv = nt * 48;
           mbar_expect_tx(&st_full[s], bk + bs + bv);
-          unsigned char* st = sm + Sm::kOffStage + s * ((Sm::kStageBytes + 1023) / 1024) * 1024;
+          unsigned char* st = sm + s * Sm::kStageStride;
           bulk_g2s(st, a.kidx + (row0 + t0) * kRbk, bk, &st_full[s]);
           bulk_g2s(st + kTT * kRbk, a.ksign + (row0 + t0) * 4, bs, &st_full[s]);
           bulk_g2s(st + kTT * (kRbk + 16), a.vidx + (row0 + t0) * 48, bv, &st_full[s]);
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id_s = idesc_i8(false), id_v = idesc_i8(true);
+      const uint32_t id_mse = idesc_i8(true, false), id_sgn = idesc_i8(false, false), id_v = idesc_i8(true, true);
       const uint64_t p_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffP));
       const uint64_t b_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffB));
       const uint64_t vh_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffVh));
@@ -352,21 +352,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         if (ns < total) {
           const int b = ns & 1;
           const int ib = s_k & 1;
-          if (mbar_try_wait(&b_full[ib], (s_k >> 1) & 1) && mbar_try_wait(a_full, ns & 1) &&
+          if (mbar_try_wait(&b_full[ib], (s_k >> 1) & 1) && mbar_try_wait(&a_full[b], (ns >> 1) & 1) &&
               mbar_try_wait(&ds_free[b], ((ns >> 1) & 1) ^ 1)) {
             tc_fence_after();
-            const uint32_t d = tmem + kColDs + b * kDsCols;
-            const uint64_t bq = b_desc0 + ((ib * 4096) >> 4), bsg = b_desc0 + ((ib * 4096 + 2048) >> 4);
+            const uint32_t d = tmem + kColDs + b * 32;
+            const uint32_t a0 = tmem + kColA + b * 128;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {       // a1, a2, a3 against q limbs; sign bytes against s limbs
+            for (int ch = 0; ch < 3; ++ch) {       // a1, a2, a3 against B1, B2, B3 (limb-shifted q)
+              const uint64_t bq = b_desc0 + (((ib * 4 + ch) * 2048) >> 4);
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t bd = (ch == 3 ? bsg : bq) + ((k * 32) >> 4);
-                umma_i8_ts(d + ch * 16, tmem + kColA + ch * 32 + k * 8, bd, id_s, k != 0);
-              }
+              for (int k = 0; k < 4; ++k) umma_i8_ts(d, a0 + ch * 32 + k * 8, bq + ((k * 32) >> 4), id_mse, (ch | k) != 0);
             }
+            const uint64_t bs = b_desc0 + (((ib * 4 + 3) * 2048) >> 4);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) umma_i8_ts(d + 16, a0 + 96 + k * 8, bs + ((k * 32) >> 4), id_sgn, k != 0);
             umma_commit(&s_full[b]);
-            umma_commit(a_free);
+            umma_commit(&a_free[b]);
             ++ns;
             if (--s_left == 0) {           // next item of this CTA
               s_item += gridDim.x;
@@ -411,11 +412,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
       }
     }
   } else if (warp < 6) {
-    // ----------------------------------------------- WG A: key dequantisation
-    const int t = tid - 64;                       // token within the tile = TMEM lane
+    // ------------------------------------------------- key operands (TMEM)
     const int q = warp & 3;                       // lane quadrant (warps 2..5 -> 2,3,0,1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const int row = q * 32 + lane;                // TMEM lane this thread writes
+    const int row = q * 32 + lane;                // token = TMEM lane this thread writes
     uint32_t k1[4], k2[4], k3[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -423,20 +423,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
       k2[u] = tab[4 + u];
       k3[u] = tab[8 + u];
     }
-    (void)t;
     int j = 0;
-    for (int item = blockIdx.x; item < A.n_items; item += gridDim.x) {
+    bool stop = false;
+    for (int item = blockIdx.x; !stop && item < A.n_items; item += gridDim.x) {
       int64_t tb, te;
       const int nt_tiles = item_tiles(item, tb, te);
-      bool stop = false;
       for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
         const int s = j % kStages;
+        const int b = j & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&st_full[s], (j / kStages) & 1))) {
           if (lane == 0) fail();
           stop = true;
           break;
         }
-        const unsigned char* st = sm + Sm::kOffStage + s * ((Sm::kStageBytes + 1023) / 1024) * 1024;
+        const unsigned char* st = sm + s * Sm::kStageStride;
         uint32_t w[kRbk / 4 + 1];
 #pragma unroll
         for (int u = 0; u < kRbk / 16; ++u) {
@@ -447,67 +447,62 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         const uint4 sg = reinterpret_cast<const uint4*>(st + kTT * kRbk + row * 16)[0];
         __syncwarp();
         if (lane == 0) mbar_arrive(&st_empty[s]);
-        if (!__all_sync(0xffffffffu, mbar_wait(a_free, (j & 1) ^ 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&a_free[b], ((j >> 1) & 1) ^ 1))) {
           if (lane == 0) fail();
           stop = true;
           break;
         }
         tc_fence_after();
-        const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w};
+        const uint32_t acol = lane_addr + kColA + b * 128;
+        // Nibble selectors of the 128 codes: word g holds codes 8g..8g+7.
+        uint32_t nib[16];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {           // 32 coordinates per chunk
-          uint32_t v1[8], v2[8], v3[8], vb[8];
+        for (int g = 0; g < 16; ++g) {
+          const int off = KB * g;                 // byte offset of the group
+          const int wi = off >> 2, shf = 8 * (off & 3);
+          const uint32_t x = shf == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], shf);
+          if (KB == 3) nib[g] = nibbles3(x);
+          else if (KB == 2) nib[g] = nibbles2(x);
+          else nib[g] = x;                        // 4-bit codes are nibbles already
+        }
+        uint32_t v[32];
 #pragma unroll
-          for (int g2 = 0; g2 < 4; ++g2) {          // 8 codes per group
-            const int g = ch * 4 + g2;
-            const int off = KB * g;                 // byte offset of the group
-            const int wi = off >> 2, shf = 8 * (off & 3);
-            const uint32_t x = shf == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], shf);
-            uint32_t lo = 0u, hi = 0u;
-            if (KB == 3) {
-              spread3(x, lo, hi);
-            } else if (KB == 2) {
-              spread2(x, lo, hi);
-            }
+        for (int limb = 0; limb < 3; ++limb) {
+          const uint32_t(&t)[4] = limb == 0 ? k1 : (limb == 1 ? k2 : k3);
+#pragma unroll
+          for (int g = 0; g < 16; ++g) {
             if (KB <= 3) {
-              v1[2 * g2] = prmt(k1[0], k1[1], lo);
-              v1[2 * g2 + 1] = prmt(k1[0], k1[1], hi);
-              v2[2 * g2] = prmt(k2[0], k2[1], lo);
-              v2[2 * g2 + 1] = prmt(k2[0], k2[1], hi);
-              v3[2 * g2] = prmt(k3[0], k3[1], lo);
-              v3[2 * g2 + 1] = prmt(k3[0], k3[1], hi);
-            } else {                                // 4-bit codes: nibbles already
-              v1[2 * g2] = lut16(k1, x & 0xFFFFu);
-              v1[2 * g2 + 1] = lut16(k1, x >> 16);
-              v2[2 * g2] = lut16(k2, x & 0xFFFFu);
-              v2[2 * g2 + 1] = lut16(k2, x >> 16);
-              v3[2 * g2] = lut16(k3, x & 0xFFFFu);
-              v3[2 * g2 + 1] = lut16(k3, x >> 16);
+              v[2 * g] = prmt(t[0], t[1], nib[g]);
+              v[2 * g + 1] = prmt(t[0], t[1], nib[g] >> 16);
+            } else {
+              v[2 * g] = lut16(t, nib[g] & 0xFFFFu);
+              v[2 * g + 1] = lut16(t, nib[g] >> 16);
             }
           }
-#pragma unroll
-          for (int n = 0; n < 8; ++n) vb[n] = bits4_to_bytes((sgw[ch] >> (4 * n)) & 15u);
-          tmem_st8(lane_addr + kColA + 0 + ch * 8, v1);
-          tmem_st8(lane_addr + kColA + 32 + ch * 8, v2);
-          tmem_st8(lane_addr + kColA + 64 + ch * 8, v3);
-          tmem_st8(lane_addr + kColA + 96 + ch * 8, vb);
+          tmem_st32(acol + limb * 32, v);
         }
+        // Sign chunk: column 4 m + u = sign word u AND (0x01010101 << m).
+        const uint32_t sw[4] = {sg.x, sg.y, sg.z, sg.w};
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) v[4 * m + u] = sw[u] & (0x01010101u << m);
+        tmem_st32(acol + 96, v);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(a_full);
+        if (lane == 0) mbar_arrive(&a_full[b]);
       }
-      if (stop) break;
     }
   } else if (warp < 10) {
-    // --------------------------------------------- WG B: value dequantisation
+    // ------------------------------------------------ value operands (smem)
     const int row = tid - 192;                    // token within the tile
     const uint32_t v1t[2] = {tab[12], tab[13]}, v2t[2] = {tab[16], tab[17]};
     int j = 0;
-    for (int item = blockIdx.x; item < A.n_items; item += gridDim.x) {
+    bool stop = false;
+    for (int item = blockIdx.x; !stop && item < A.n_items; item += gridDim.x) {
       int64_t tb, te;
       const int nt_tiles = item_tiles(item, tb, te);
-      bool stop = false;
       for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
         const int s = j % kStages;
         const int b = j & 1;
@@ -516,7 +511,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
           stop = true;
           break;
         }
-        const unsigned char* st = sm + Sm::kOffStage + s * ((Sm::kStageBytes + 1023) / 1024) * 1024;
+        const unsigned char* st = sm + s * Sm::kStageStride;
         uint32_t w[13];
 #pragma unroll
         for (int u = 0; u < 3; ++u) {
@@ -543,12 +538,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
             const int g = 2 * c16 + h;
             const int off = 3 * g, wi = off >> 2, shf = 8 * (off & 3);
             const uint32_t x = shf == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], shf);
-            uint32_t lo, hi;
-            spread3(x, lo, hi);
-            o1[2 * h] = prmt(v1t[0], v1t[1], lo);
-            o1[2 * h + 1] = prmt(v1t[0], v1t[1], hi);
-            o2[2 * h] = prmt(v2t[0], v2t[1], lo);
-            o2[2 * h + 1] = prmt(v2t[0], v2t[1], hi);
+            const uint32_t nb = nibbles3(x);
+            o1[2 * h] = prmt(v1t[0], v1t[1], nb);
+            o1[2 * h + 1] = prmt(v1t[0], v1t[1], nb >> 16);
+            o2[2 * h] = prmt(v2t[0], v2t[1], nb);
+            o2[2 * h + 1] = prmt(v2t[0], v2t[1], nb >> 16);
           }
           const uint32_t off = atom * 1024 + r8 * 128 + ((c16 ^ r8) << 4);
           *reinterpret_cast<uint4*>(vh + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
@@ -558,15 +552,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         __syncwarp();
         if (lane == 0) mbar_arrive(&vh_full[b]);
       }
-      if (stop) break;
     }
   } else {
-    // ------------------------------------- WG C: scores, softmax, epilogues
+    // ------------------------------------- scores, softmax, value epilogue
     const int cw = warp - 10;                     // 0..3
     const int q = warp & 3;                       // lane quadrant (warps 10..13 -> 2,3,0,1)
     const int lrow = q * 32 + lane;               // TMEM lane = token / coordinate
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const float alpha = static_cast<float>(dev::kSqrtHalfPi / kD);
+    constexpr float kLog2e = 1.4426950408889634f;
     int j = 0, item_idx = 0;
     bool stop = false;
     for (int item = blockIdx.x; item < A.n_items && !stop; item += gridDim.x, ++item_idx) {
@@ -576,233 +570,245 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
       const int split = item % sh.n_splits;
       const int kv = static_cast<int>(unit % sh.hkv), bb = static_cast<int>(unit / sh.hkv);
       const int G = sh.hq / sh.hkv;
+      const int64_t row0 = item_row0(item);
       int64_t qrow[kRowsTc];
 #pragma unroll
       for (int r = 0; r < kRowsTc; ++r)
         qrow[r] = (int64_t(bb) * sh.hq + kv * G + r / sh.nq) * sh.nq + r % sh.nq;
-      // B operands of this item: rows (r, limb) of q_rot and s as int8, K-major.
+      // ---- item prologue: row scales, the item's largest ||v||, B tiles.
       const int ib = item_idx & 1;
-      unsigned char* bq = sm + Sm::kOffB + ib * 4096;
-      float* isc = item_scale + ib * 16;          // sq[4] | ss[4] | ssum[4]
+      float qv[kRowsTc], sv[kRowsTc];
+      float sq[kRowsTc], ss[kRowsTc], ssum[kRowsTc];
       {
-        // ct = coordinate i: row scales first (max |q_r|, max |s_r| over i).
-        float qv[kRowsTc], sv[kRowsTc];
+        const float jscale = __uint_as_float(static_cast<uint32_t>(127 - (lrow & 7)) << 23);   // 2^-(i mod 8)
+        float loc[12];
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
           qv[r] = a.qs[qrow[r] * 2 * kD + lrow];
           sv[r] = a.qs[qrow[r] * 2 * kD + kD + lrow];
+          loc[r] = fabsf(qv[r]);
+          loc[4 + r] = fabsf(sv[r]) * jscale;
+          loc[8 + r] = sv[r];
+        }
+#pragma unroll
+        for (int u = 0; u < 12; ++u) {
+          const float x = (u >= 8 && u < 12) ? warp_sum(loc[u]) : warp_max(loc[u]);
+          if (lane == 0) red[cw * 16 + u] = x;
+        }
+        wg_sync(1);
+        float tot[12];
+#pragma unroll
+        for (int u = 0; u < 12; ++u) {
+          float x = red[u];
+#pragma unroll
+          for (int w2 = 1; w2 < 4; ++w2) x = (u >= 8 && u < 12) ? x + red[w2 * 16 + u] : fmaxf(x, red[w2 * 16 + u]);
+          tot[u] = x;
         }
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          const float mq = warp_max(fabsf(qv[r])), ms = warp_max(fabsf(sv[r]));
-          const float ssum = warp_sum(sv[r]);
-          if (lane == 0) {
-            red[cw * 8 + r] = mq;
-            red[cw * 8 + 4 + r] = ms;
-            scr[cw * 4 + r] = ssum;
-          }
+          sq[r] = tot[r] > 0.f ? tot[r] / 127.f : 1.f;
+          ss[r] = tot[4 + r] > 0.f ? tot[4 + r] / 127.f : 1.f;
+          ssum[r] = tot[8 + r];
         }
-        wg_sync(2);
-        float sq[kRowsTc], ss[kRowsTc];
+        // B tiles: B1/B2/B3 rows 4 r + w hold limb w, w-1, w-2 of q_rot row r;
+        // Bs rows 4 r + l hold limb l of s' at K position 16 (i mod 8) + i / 8.
+        unsigned char* bt = sm + Sm::kOffB + ib * 4 * 2048;
+        const int ks = 16 * (lrow & 7) + (lrow >> 3);
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          float mq = 0.f, ms = 0.f, su = 0.f;
+          int lq[4], ls[4];
+          limbs4(qv[r] / sq[r], lq);
+          limbs4(sv[r] * jscale / ss[r], ls);
 #pragma unroll
           for (int w2 = 0; w2 < 4; ++w2) {
-            mq = fmaxf(mq, red[w2 * 8 + r]);
-            ms = fmaxf(ms, red[w2 * 8 + 4 + r]);
-            su += scr[w2 * 4 + r];
+            bt[sw_byte(4 * r + w2, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(lq[w2]));
+            bt[2048 + sw_byte(4 * r + w2, lrow)] =
+                static_cast<unsigned char>(static_cast<int8_t>(w2 >= 1 ? lq[w2 - 1] : 0));
+            bt[4096 + sw_byte(4 * r + w2, lrow)] =
+                static_cast<unsigned char>(static_cast<int8_t>(w2 >= 2 ? lq[w2 - 2] : 0));
+            bt[6144 + sw_byte(4 * r + w2, ks)] = static_cast<unsigned char>(static_cast<int8_t>(ls[w2]));
           }
-          sq[r] = mq > 0.f ? mq / 127.f : 1.f;
-          ss[r] = ms > 0.f ? ms / 127.f : 1.f;
-          if (lrow == 0) {
-            isc[r] = sq[r];
-            isc[4 + r] = ss[r];
-            isc[8 + r] = su;
-          }
-        }
-        // Write limbs: B row n = 3 r + l holds limb l of row r over coordinates.
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          int l0, l1, l2;
-          limbs3(qv[r], 1.f / sq[r], l0, l1, l2);
-          bq[sw_byte(3 * r + 0, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l0));
-          bq[sw_byte(3 * r + 1, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l1));
-          bq[sw_byte(3 * r + 2, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l2));
-          limbs3(sv[r], 1.f / ss[r], l0, l1, l2);
-          bq[2048 + sw_byte(3 * r + 0, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l0));
-          bq[2048 + sw_byte(3 * r + 1, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l1));
-          bq[2048 + sw_byte(3 * r + 2, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l2));
-        }
-        // Rows 12..15 are zero.
-#pragma unroll
-        for (int n = 12; n < 16; ++n) {
-          bq[sw_byte(n, lrow)] = 0;
-          bq[2048 + sw_byte(n, lrow)] = 0;
         }
         fence_proxy_async_smem();
-        wg_sync(2);
         __syncwarp();
         if (lane == 0) mbar_arrive(&b_full[ib]);
       }
-      float m_run[kRowsTc], l_run[kRowsTc], acc[kRowsTc];
+      float kq[kRowsTc], ks2[kRowsTc];
+#pragma unroll
+      for (int r = 0; r < kRowsTc; ++r) {
+        kq[r] = a.scale * k_scale * sq[r];
+        ks2[r] = 2.f * ss[r];
+      }
+      float m_run[kRowsTc], l_part[kRowsTc], acc[kRowsTc];
+      float corr_prev[kRowsTc], sp_prev[kRowsTc];       // of the tile whose values fold next
 #pragma unroll
       for (int r = 0; r < kRowsTc; ++r) {
         m_run[r] = -INFINITY;
-        l_run[r] = 0.f;
+        l_part[r] = 0.f;
         acc[r] = 0.f;
+        corr_prev[r] = 0.f;
+        sp_prev[r] = 1.f;
       }
-      const int64_t row0 = item_row0(item);
-      // Value epilogue of tile jj (this thread = coordinate ct).
+      // Value epilogue of tile jj (this thread = coordinate lrow).
       auto value_epilogue = [&](int jj) -> bool {
-        const int bb2 = jj & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_full[bb2], (jj >> 1) & 1))) return false;
+        const int b2 = jj & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_full[b2], (jj >> 1) & 1))) return false;
         tc_fence_after();
         uint32_t d[32];
-        uint32_t d0[16], d1[16];
-        tmem_ld16(lane_addr + kColDo + bb2 * 32, d0);
-        tmem_ld16(lane_addr + kColDo + bb2 * 32 + 16, d1);
+        tmem_ld32(lane_addr + kColDo + b2 * 32, d);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&do_free[bb2]);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          d[u] = d0[u];
-          d[16 + u] = d1[u];
-        }
-        const float* rg = ring + bb2 * 8;
+        if (lane == 0) mbar_arrive(&do_free[b2]);
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          // column (r, limb) = 2 r + limb in each value-limb chain
-          const float hi = static_cast<float>(static_cast<int>(d[2 * r])) +
-                           static_cast<float>(static_cast<int>(d[2 * r + 1])) * (1.f / 128.f);
-          const float lo = static_cast<float>(static_cast<int>(d[16 + 2 * r])) +
-                           static_cast<float>(static_cast<int>(d[16 + 2 * r + 1])) * (1.f / 128.f);
-          acc[r] = acc[r] * rg[r] + v_scale * rg[4 + r] * (hi + lo * (1.f / 128.f));
+          // column (r, weight limb) = 2 r + limb in each value-limb chain
+          const float hi = fmaf(static_cast<float>(static_cast<int>(d[2 * r + 1])), 1.f / 128.f,
+                                static_cast<float>(static_cast<int>(d[2 * r])));
+          const float lo = fmaf(static_cast<float>(static_cast<int>(d[16 + 2 * r + 1])), 1.f / 128.f,
+                                static_cast<float>(static_cast<int>(d[16 + 2 * r])));
+          acc[r] = fmaf(acc[r], corr_prev[r], v_scale * sp_prev[r] * fmaf(lo, 1.f / 128.f, hi));
         }
         return true;
       };
+      // Norms of the next tile are loaded one tile ahead.
+      float kn_n = 0.f, rn_n = 0.f, vn_n = 0.f;
+      if (lrow < te - tb) {
+        kn_n = __ldg(a.knorm + row0 + tb + lrow);
+        rn_n = __ldg(a.krnorm + row0 + tb + lrow);
+        vn_n = __ldg(a.vnorm + row0 + tb + lrow);
+      }
       for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
         const int b = j & 1;
         const int64_t t0 = tb + int64_t(tj) * kTT;
         const int nt = static_cast<int>((te - t0 < kTT) ? te - t0 : kTT);
         const bool valid = lrow < nt;
-        float kn = 0.f, rn = 0.f, vn = 0.f;
-        if (valid) {
-          kn = __ldg(a.knorm + row0 + t0 + lrow);
-          rn = __ldg(a.krnorm + row0 + t0 + lrow);
-          vn = __ldg(a.vnorm + row0 + t0 + lrow);
+        const float kn = kn_n, rn = rn_n, vn = vn_n;
+        if (t0 + kTT + lrow < te) {
+          kn_n = __ldg(a.knorm + row0 + t0 + kTT + lrow);
+          rn_n = __ldg(a.krnorm + row0 + t0 + kTT + lrow);
+          vn_n = __ldg(a.vnorm + row0 + t0 + kTT + lrow);
         }
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1));
         tc_fence_after();
-        uint32_t d0[16], d1[16], d2[16], d3[16];
-        tmem_ld16(lane_addr + kColDs + b * kDsCols, d0);
-        tmem_ld16(lane_addr + kColDs + b * kDsCols + 16, d1);
-        tmem_ld16(lane_addr + kColDs + b * kDsCols + 32, d2);
-        tmem_ld16(lane_addr + kColDs + b * kDsCols + 48, d3);
+        uint32_t d[32];
+        tmem_ld32(lane_addr + kColDs + b * 32, d);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ds_free[b]);
         float score[kRowsTc];
+        bool need = false;
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          float c1 = 0.f, c2 = 0.f, c3 = 0.f, sb = 0.f;
-#pragma unroll
-          for (int l = 2; l >= 0; --l) {
-            c1 = c1 * (1.f / 128.f) + static_cast<float>(static_cast<int>(d0[3 * r + l]));
-            c2 = c2 * (1.f / 128.f) + static_cast<float>(static_cast<int>(d1[3 * r + l]));
-            c3 = c3 * (1.f / 128.f) + static_cast<float>(static_cast<int>(d2[3 * r + l]));
-            sb = sb * (1.f / 128.f) + static_cast<float>(static_cast<int>(d3[3 * r + l]));
-          }
-          const float mse = k_scale * isc[r] * (c1 + (c2 + c3 * (1.f / 128.f)) * (1.f / 128.f));
-          const float qjl = 2.f * isc[4 + r] * sb - isc[8 + r];
-          score[r] = valid ? a.scale * (kn * mse + alpha * rn * qjl) : -INFINITY;
+          const float mse = limb_sum4(d + 4 * r);
+          const float sgn = limb_sum4(d + 16 + 4 * r);
+          const float qjl = fmaf(ks2[r], sgn, -ssum[r]);
+          score[r] = valid ? fmaf(kq[r] * kn, mse, a.scale * alpha * rn * qjl) : -INFINITY;
+          need |= score[r] > m_run[r];
         }
         if (a.scores_out && valid) {
 #pragma unroll
           for (int r = 0; r < kRowsTc; ++r) a.scores_out[qrow[r] * sh.n_ctx + t0 + lrow] = score[r];
         }
-        // Online softmax over the tile.
+        // Per-warp maxima of z = score log2 e + log2 ||v|| (the largest weight
+        // p ||v|| of the tile, up to the running maximum), published before the
+        // vote barrier; slots alternate by tile parity.
+        {
+          const float lv = valid ? __log2f(vn) : -INFINITY;
 #pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          const float mx = warp_max(score[r]);
-          if (lane == 0) red[cw * 8 + r] = mx;
-        }
-        if (wg_sync_or(3, !ok || *abort_s != 0)) {
-          if (!ok && lane == 0 && cw == 0) fail();
-          stop = true;
-          break;
-        }
-        float corr[kRowsTc], p[kRowsTc];
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          float mx = red[r];
-#pragma unroll
-          for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, red[w2 * 8 + r]);
-          const float m_new = fmaxf(m_run[r], mx);
-          corr[r] = (m_run[r] == -INFINITY) ? 0.f : __expf(m_run[r] - m_new);
-          m_run[r] = m_new;
-          p[r] = valid ? __expf(score[r] - m_new) : 0.f;
-        }
-        wg_sync(2);                                // everyone has read the maxima
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          const float ps = warp_sum(p[r]);
-          const float wm = warp_max(p[r] * vn);
-          if (lane == 0) {
-            red[cw * 8 + r] = ps;
-            red[cw * 8 + 4 + r] = wm;
+          for (int r = 0; r < kRowsTc; ++r) {
+            const float zm = warp_max(valid ? fmaf(score[r], kLog2e, lv) : -INFINITY);
+            if (lane == 0) zred[(b * 4 + cw) * 4 + r] = zm;
           }
         }
-        wg_sync(2);
-        float sp[kRowsTc];
+        float corr[kRowsTc];
+#pragma unroll
+        for (int r = 0; r < kRowsTc; ++r) corr[r] = 1.f;
+        // The running maximum moves only when some score of the tile exceeds it.
+        if (wg_sync_or(1, need || !ok || *abort_s != 0)) {
+          if (wg_sync_or(1, !ok || *abort_s != 0)) {
+            if (!ok && lane == 0 && cw == 0) fail();
+            stop = true;
+            break;
+          }
+#pragma unroll
+          for (int r = 0; r < kRowsTc; ++r) {
+            const float mx = warp_max(score[r]);
+            if (lane == 0) red[cw * 16 + r] = mx;
+          }
+          wg_sync(1);
+#pragma unroll
+          for (int r = 0; r < kRowsTc; ++r) {
+            float mx = red[r];
+#pragma unroll
+            for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, red[w2 * 16 + r]);
+            const float m_new = fmaxf(m_run[r], mx);
+            corr[r] = (m_run[r] == -INFINITY) ? 0.f : exp2f((m_run[r] - m_new) * kLog2e);
+            l_part[r] *= corr[r];
+            m_run[r] = m_new;
+          }
+        }
+        // Weight scale of each row: max_t p ||v|| / 127, with a margin so the
+        // largest limb stays at or below 127 after rounding.
+        float inv_sp[kRowsTc], sp_cur[kRowsTc];
+        {
+          const float4* zr = reinterpret_cast<const float4*>(zred + b * 16);
+          const float4 z0 = zr[0], z1 = zr[1], z2 = zr[2], z3 = zr[3];
+          const float zmax[kRowsTc] = {fmaxf(fmaxf(z0.x, z1.x), fmaxf(z2.x, z3.x)),
+                                       fmaxf(fmaxf(z0.y, z1.y), fmaxf(z2.y, z3.y)),
+                                       fmaxf(fmaxf(z0.z, z1.z), fmaxf(z2.z, z3.z)),
+                                       fmaxf(fmaxf(z0.w, z1.w), fmaxf(z2.w, z3.w))};
+#pragma unroll
+          for (int r = 0; r < kRowsTc; ++r) {
+            float wmax = exp2f(zmax[r] - m_run[r] * kLog2e) * (1.f + 1.f / 4096.f);
+            if (!(wmax > 0.f)) wmax = 127.f;           // no weight in this tile (all ||v|| = 0)
+            sp_cur[r] = wmax * (1.f / 127.f);
+            inv_sp[r] = 127.f / wmax;
+          }
+        }
+        float p[kRowsTc];
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          float ps = 0.f, wm = 0.f;
-#pragma unroll
-          for (int w2 = 0; w2 < 4; ++w2) {
-            ps += red[w2 * 8 + r];
-            wm = fmaxf(wm, red[w2 * 8 + 4 + r]);
-          }
-          l_run[r] = l_run[r] * corr[r] + ps;
-          sp[r] = wm > 0.f ? wm / 127.f : 1.f;
-        }
-        // Publish this tile's correction and weight scale for its value epilogue.
-        if (lrow < kRowsTc) {
-#pragma unroll
-          for (int r = 0; r < kRowsTc; ++r)
-            if (r == lrow) {
-              ring[b * 8 + r] = corr[r];
-              ring[b * 8 + 4 + r] = sp[r];
-            }
+          p[r] = valid ? exp2f((score[r] - m_run[r]) * kLog2e) : 0.f;
+          l_part[r] += p[r];
         }
         // Weight limbs into the P tile (row 2 r + limb, column = token).
         if (!__all_sync(0xffffffffu, mbar_wait(&p_free[b], ((j >> 1) & 1) ^ 1)) && lane == 0) fail();
         unsigned char* pt = sm + Sm::kOffP + b * 2048;
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          const float x = p[r] * vn / sp[r];
+          const float x = fminf(p[r] * vn * inv_sp[r], 127.f);
           const int l0 = __float2int_rn(x);
           const int l1 = __float2int_rn((x - static_cast<float>(l0)) * 128.f);
           pt[sw_byte(2 * r, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l0));
           pt[sw_byte(2 * r + 1, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l1));
         }
-#pragma unroll
-        for (int n = 8; n < 16; ++n) pt[sw_byte(n, lrow)] = 0;
         fence_proxy_async_smem();
-        wg_sync(2);                                // ring + red reads done before reuse
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
         // Fold the previous tile's values (its correction comes first).
         if (tj >= 1 && !value_epilogue(j - 1)) {
           if (lane == 0) fail();
         }
+#pragma unroll
+        for (int r = 0; r < kRowsTc; ++r) {
+          corr_prev[r] = corr[r];
+          sp_prev[r] = sp_cur[r];
+        }
       }
       if (stop) break;
       // Last tile of the item, then the partials.
       if (!value_epilogue(j - 1) && lane == 0) fail();
+      float lsum[kRowsTc];
+#pragma unroll
+      for (int r = 0; r < kRowsTc; ++r) {
+        const float x = warp_sum(l_part[r]);
+        if (lane == 0) red2[cw * 4 + r] = x;
+      }
+      wg_sync(1);
+#pragma unroll
+      for (int r = 0; r < kRowsTc; ++r) lsum[r] = red2[r] + red2[4 + r] + red2[8 + r] + red2[12 + r];
       const int64_t pbase = (int64_t(split)) * (kD + 2);
 #pragma unroll
       for (int r = 0; r < kRowsTc; ++r) {
@@ -810,7 +816,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         pr[lrow] = acc[r];
         if (lrow == 0) {
           pr[kD] = m_run[r];
-          pr[kD + 1] = l_run[r];
+          pr[kD + 1] = lsum[r];
         }
       }
     }
