@@ -65,13 +65,16 @@ DecodeShape make_shape(const tq_layout* L, int batch, int hq, int hkv, int nq, i
   const int64_t per = (tiles + splits - 1) / splits;
   s.chunk = per * kT;
   s.n_splits = static_cast<int>((n_ctx + s.chunk - 1) / s.chunk);
+  s.n_parts = s.n_splits;
   s.n_rows = int64_t(batch) * hq * nq;
   return s;
 }
 
 size_t shape_workspace_bytes(const DecodeShape& s) {
   const size_t qs = size_t(s.n_rows) * 2 * s.d * sizeof(float);
-  const size_t part = size_t(s.n_rows) * s.n_splits * (s.d + 2) * sizeof(float);
+  // Room for two partial records per split (the tensor-core kernel splits each
+  // work item into its even and odd tiles).
+  const size_t part = size_t(s.n_rows) * 2 * s.n_splits * (s.d + 2) * sizeof(float);
   return ((qs + 255) / 256) * 256 + part;
 }
 
@@ -400,11 +403,11 @@ __global__ void __launch_bounds__(kT) decode_main(DecodeArgs a) {
     const int i = tid + c * kT;
     if (i < D) {
 #pragma unroll
-      for (int r = 0; r < R; ++r) a.part[(qrow(r) * sh.n_splits + split) * (D + 2) + i] = acc[c][r];
+      for (int r = 0; r < R; ++r) a.part[(qrow(r) * sh.n_parts + split) * (D + 2) + i] = acc[c][r];
     }
   }
   if (tid < R) {
-    float* p = a.part + (qrow(tid) * sh.n_splits + split) * (D + 2);
+    float* p = a.part + (qrow(tid) * sh.n_parts + split) * (D + 2);
     p[D] = s.m[tid];
     p[D + 1] = s.l[tid];
   }
@@ -417,7 +420,7 @@ template <int RPG>
 __global__ void __launch_bounds__(kBlkThreads) decode_combine(DecodeArgs a, RowBlocks rb) {
   extern __shared__ __align__(16) float blk_smem[];
   const DecodeShape& s = a.sh;
-  const int d = s.d, ns = s.n_splits;
+  const int d = s.d, ns = s.n_parts;
   float* Ms = blk_smem;                       // [d][d+1] Pi_V
   float* os = Ms + d * (d + 1);               // [d][16] merged rotated outputs
   float* wl = os + d * kBlkRows;              // [16] 1 / L per row; [16] max per row
@@ -631,6 +634,7 @@ extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q,
     const char* path = std::getenv("TQ_DECODE_PATH");
     const bool cuda_core = path && (std::strcmp(path, "v1") == 0 || std::strcmp(path, "v2") == 0);
     if (!cuda_core && tc_decode_supported(a)) {
+      a.sh.n_parts = 2 * a.sh.n_splits;
       e = tc_decode_launch(a, s);
     } else {
     switch (d) {

@@ -21,22 +21,25 @@
 //           0, 1, 2, so D column 4 r + w holds sum_{l+m=w} a_l q_m.
 //   values  O[i][n] = sum_t c_V[code_ti] w_t,n: A (smem, M-major) the value
 //           codebook as two int8 limbs per coordinate, one 128-byte row per
-//           token; B the tile's weights w = p ||v|| / s_tile as two int8 limbs
-//           per query row, s_tile = max_t p ||v|| / 127 of that row, found as
-//           2^(max_t z_t - m log2 e) with z = score log2 e + log2 ||v||.
+//           token; B the tile's weights w = p ||v|| / s_item as three int8
+//           limbs per query row, s_item = max ||v|| over the work item / 127
+//           (p <= 1 because the running maximum only grows).
 // Online softmax: the running maximum per row only moves when a score of the
 // tile exceeds it (a vote over the softmax warps; the tile maximum is reduced
-// only then); the per-warp maxima of z are published before the same vote
-// barrier, so an ordinary tile costs one barrier. l is kept per thread and
-// summed once per work item; corrections and scales are uniform across the
-// softmax threads and stay in registers.
-// Roles (448 threads, one persistent CTA per SM):
+// only then), so an ordinary tile costs one barrier; l is kept per thread and
+// summed once per work item. The value warps fold each PV product into their
+// accumulators (thread = coordinate) with the tile's correction, which the
+// softmax warps leave in a four-slot ring.
+// Roles (480 threads, one persistent CTA per SM):
 //   warp 0     bulk copies of the packed index / sign planes into a 3-stage ring
-//   warp 1     TMEM owner and single-thread tcgen05.mma issuer
+//   warp 1     TMEM owner and single-thread issuer of the score MMAs
+//   warp 14    single-thread issuer of the PV MMAs
 //   warps 2-5  key operand generation into TMEM        (thread = token)
 //   warps 6-9  value operand generation into smem      (thread = token)
-//   warps 10-13 scores, softmax and weight limbs       (thread = token),
-//             the value epilogue                       (thread = coordinate)
+//             and the value epilogue                   (thread = coordinate)
+//   warps 10-13 scores, softmax and weight limbs       (thread = token); the
+//             even and odd tiles of a work item keep separate running maxima
+//             and sums, so a work item leaves two partial records
 // Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT and the CTA
 // drains its copies and MMAs before it frees TMEM and returns.
 #include <cuda.h>
@@ -57,7 +60,7 @@ using dev::warp_sum;
 constexpr int kD = 128;
 constexpr int kTT = 128;               // tokens per tile
 constexpr int kStages = 3;
-constexpr int kThreadsTc = 448;        // 14 warps
+constexpr int kThreadsTc = 480;        // 15 warps
 constexpr int kRowsTc = 4;
 
 // TMEM columns (32-bit): A_score x2 at 0, 128 (a1 | a2 | a3 | sgn, 32 each);
@@ -80,12 +83,12 @@ struct TcSm {
   static constexpr int kOffP = kOffVh + 2 * kVhBytes;               // 2 x [16 rows x 128 B]
   static constexpr int kOffB = kOffP + 2 * 2048;                    // 2 items x (B1 | B2 | B3 | Bs)
   static constexpr int kOffBar = kOffB + 2 * 4 * 2048;
-  static constexpr int kNumBars = 2 * kStages + 2 * 11 + 1;
+  static constexpr int kNumBars = 2 * kStages + 2 * 11 + 2;
   static constexpr int kOffMisc = ((kOffBar + kNumBars * 8 + 15) / 16) * 16;
-  static constexpr int kOffZ = kOffMisc + 16;                       // [2 tiles][4 warps][4] max z
-  static constexpr int kOffRed = kOffZ + 2 * 4 * 4 * 4;             // [4 warps][16]
-  static constexpr int kOffRed2 = kOffRed + 4 * 16 * 4;             // [4 warps][4]
-  static constexpr int kOffTab = kOffRed2 + 4 * 4 * 4;              // ka1 ka2 ka3 va1 va2 (4 words) + 2 scales
+  static constexpr int kOffRing = kOffMisc + 16;                    // [4 tiles][8]: corr[4], scale
+  static constexpr int kOffRed = kOffRing + 4 * 8 * 4;              // [2 groups][4 warps][16]
+  static constexpr int kOffRed2 = kOffRed + 2 * 4 * 16 * 4;         // [2 groups][4 warps][4]
+  static constexpr int kOffTab = kOffRed2 + 2 * 4 * 4 * 4;          // ka1 ka2 ka3 va1 va2 (4 words) + 2 scales
   static constexpr int kBytes = kOffTab + 22 * 4 + 1024;
 };
 
@@ -199,11 +202,22 @@ __device__ __forceinline__ void limbs4(float x, int (&l)[4]) {
     x = (x - static_cast<float>(l[u])) * 128.f;
   }
 }
+// int32 accumulator -> float, exact for |x| < 2^22 (every accumulator here:
+// at most 3 limb products of 128 terms, first limbs <= 127, others <= 64).
+__device__ __forceinline__ float i2f(uint32_t x) { return __uint_as_float(x + 0x4B400000u) - 12582912.f; }
 __device__ __forceinline__ float limb_sum4(const uint32_t* d) {
-  float v = static_cast<float>(static_cast<int>(d[3]));
-  v = fmaf(v, 1.f / 128.f, static_cast<float>(static_cast<int>(d[2])));
-  v = fmaf(v, 1.f / 128.f, static_cast<float>(static_cast<int>(d[1])));
-  return fmaf(v, 1.f / 128.f, static_cast<float>(static_cast<int>(d[0])));
+  float v = i2f(d[3]);
+  v = fmaf(v, 1.f / 128.f, i2f(d[2]));
+  v = fmaf(v, 1.f / 128.f, i2f(d[1]));
+  return fmaf(v, 1.f / 128.f, i2f(d[0]));
+}
+__device__ __forceinline__ float limb_sum3(const uint32_t* d) {
+  return fmaf(fmaf(i2f(d[2]), 1.f / 128.f, i2f(d[1])), 1.f / 128.f, i2f(d[0]));
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <int KB>
@@ -217,20 +231,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
   uint64_t* st_full = bars;                       // [3]
   uint64_t* st_empty = bars + kStages;            // [3]
   uint64_t* a_full = bars + 2 * kStages;          // [2]
-  uint64_t* a_free = a_full + 2;                  // [2]
+  uint64_t* a_free = a_full + 2;                  // [2] (aliased below)
   uint64_t* s_full = a_free + 2;                  // [2]
   uint64_t* ds_free = s_full + 2;                 // [2]
   uint64_t* vh_full = ds_free + 2;                // [2]
-  uint64_t* vh_free = vh_full + 2;                // [2]
+  uint64_t* vh_free = vh_full + 2;                // [2] (aliased below)
   uint64_t* p_full = vh_free + 2;                 // [2]
-  uint64_t* p_free = p_full + 2;                  // [2]
+  uint64_t* p_free = p_full + 2;                  // [2] (aliased below)
   uint64_t* pv_full = p_free + 2;                 // [2]
   uint64_t* do_free = pv_full + 2;                // [2]
   uint64_t* b_full = do_free + 2;                 // [2] per item parity
-  uint64_t* drain = b_full + 2;                   // [1]
+  uint64_t* drain = b_full + 2;                   // [2] score issuer, PV issuer
+  // One completion event each: the score MMAs of a tile free its key operands
+  // and fill its score columns; the PV MMAs free the value operands and the
+  // weight tile and fill the value columns.
+  a_free = s_full;
+  vh_free = pv_full;
+  p_free = pv_full;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Sm::kOffMisc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + Sm::kOffMisc + 4);
-  float* zred = reinterpret_cast<float*>(sm + Sm::kOffZ);             // [2][4 warps][4]
+  float* ring = reinterpret_cast<float*>(sm + Sm::kOffRing);          // [4][8]
   float* red = reinterpret_cast<float*>(sm + Sm::kOffRed);            // [4 warps][16]
   float* red2 = reinterpret_cast<float*>(sm + Sm::kOffRed2);          // [4 warps][4]
   uint32_t* tab = reinterpret_cast<uint32_t*>(sm + Sm::kOffTab);      // ka1 ka2 ka3 va1 va2 (4 words each)
@@ -257,8 +277,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
       mbar_init(&do_free[b], 4);
       mbar_init(&b_full[b], 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_s = 0;
+    for (int k = 0; k < 4; ++k) reinterpret_cast<int*>(sm + Sm::kOffRing)[k * 8 + 5] = -1;
     mbar_fence_init();
   }
   if (tid == 32) {
@@ -269,10 +291,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
     tmem_alloc(tmem_base_s, kTmemColsTc);
     tmem_relinquish();
   }
-  // Rows 8-15 of both weight tiles stay zero (only 2 limbs x 4 rows are used).
-  for (int e = tid; e < 2 * 1024 / 16; e += kThreadsTc) {
-    const int b = e / 64, o = e % 64;
-    reinterpret_cast<uint4*>(sm + Sm::kOffP + b * 2048 + 1024)[o] = make_uint4(0u, 0u, 0u, 0u);
+  // Rows 12-15 of both weight tiles stay zero (3 limbs x 4 rows are used).
+  for (int e = tid; e < 2 * 512 / 16; e += kThreadsTc) {
+    const int b = e / 32, o = e % 32;
+    reinterpret_cast<uint4*>(sm + Sm::kOffP + b * 2048 + 1536)[o] = make_uint4(0u, 0u, 0u, 0u);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -327,89 +349,66 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         mbar_wait(&st_full[jj % kStages], (jj / kStages) & 1);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 14) {
+    // ------------------------------------------ MMA issuers (one thread each)
+    // warp 1 issues the score MMAs, warp 18 the PV MMAs, so the issue
+    // latencies of the two chains overlap.
     if (lane == 0) {
       const uint32_t id_mse = idesc_i8(true, false), id_sgn = idesc_i8(false, false), id_v = idesc_i8(true, true);
       const uint64_t p_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffP));
       const uint64_t b_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffB));
       const uint64_t vh_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffVh));
-      int total = 0;
-      for (int item = blockIdx.x; item < A.n_items; item += gridDim.x) {
+      int j = 0, s_k = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < A.n_items; item += gridDim.x, ++s_k) {
         int64_t tb, te;
-        total += item_tiles(item, tb, te);
-      }
-      int ns = 0, np = 0;                 // next score tile, next PV tile
-      int s_item = blockIdx.x, s_k = 0, s_left = 0;
-      if (s_item < A.n_items) {
-        int64_t tb, te;
-        s_left = item_tiles(s_item, tb, te);
-      }
-      uint64_t last = globaltimer_ns();
-      while (np < total) {
-        if (*abort_s) break;
-        bool progress = false;
-        if (ns < total) {
-          const int b = ns & 1;
-          const int ib = s_k & 1;
-          if (mbar_try_wait(&b_full[ib], (s_k >> 1) & 1) && mbar_try_wait(&a_full[b], (ns >> 1) & 1) &&
-              mbar_try_wait(&ds_free[b], ((ns >> 1) & 1) ^ 1)) {
+        const int nt_tiles = item_tiles(item, tb, te);
+        for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
+          const int b = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          if (*abort_s) { ok = false; break; }
+          if (warp == 1) {
+            const int ib = s_k & 1;
+            if (!mbar_wait(&b_full[ib], (s_k >> 1) & 1) || !mbar_wait(&a_full[b], ph) ||
+                !mbar_wait(&ds_free[b], ph ^ 1)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d = tmem + kColDs + b * 32;
             const uint32_t a0 = tmem + kColA + b * 128;
-#pragma unroll
-            for (int ch = 0; ch < 3; ++ch) {       // a1, a2, a3 against B1, B2, B3 (limb-shifted q)
-              const uint64_t bq = b_desc0 + (((ib * 4 + ch) * 2048) >> 4);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) umma_i8_ts(d, a0 + ch * 32 + k * 8, bq + ((k * 32) >> 4), id_mse, (ch | k) != 0);
-            }
+            // a1, a2, a3 against B1, B2, B3 (limb-shifted q) into the MSE
+            // columns, the sign chunk into its own columns.
             const uint64_t bs = b_desc0 + (((ib * 4 + 3) * 2048) >> 4);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) umma_i8_ts(d + 16, a0 + 96 + k * 8, bs + ((k * 32) >> 4), id_sgn, k != 0);
-            umma_commit(&s_full[b]);
-            umma_commit(&a_free[b]);
-            ++ns;
-            if (--s_left == 0) {           // next item of this CTA
-              s_item += gridDim.x;
-              ++s_k;
-              if (s_item < A.n_items) {
-                int64_t tb, te;
-                s_left = item_tiles(s_item, tb, te);
-              }
+            for (int step = 0; step < 12; ++step) {
+              const int ch = step >> 2, k = step & 3;
+              const uint64_t bq = b_desc0 + (((ib * 4 + ch) * 2048) >> 4);
+              umma_i8_ts(d, a0 + ch * 32 + k * 8, bq + ((k * 32) >> 4), id_mse, step != 0);
+              if (step < 4) umma_i8_ts(d + 16, a0 + 96 + k * 8, bs + ((k * 32) >> 4), id_sgn, k != 0);
             }
-            progress = true;
-          }
-        }
-        if (np < ns) {
-          const int b = np & 1;
-          const uint32_t ph = (np >> 1) & 1;
-          if (mbar_try_wait(&vh_full[b], ph) && mbar_try_wait(&p_full[b], ph) &&
-              mbar_try_wait(&do_free[b], ph ^ 1)) {
+            umma_commit(&s_full[b]);
+          } else {
+            if (!mbar_wait(&vh_full[b], ph) || !mbar_wait(&p_full[b], ph) || !mbar_wait(&do_free[b], ph ^ 1)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const uint32_t d = tmem + kColDo + b * 32;
             const uint64_t pb = p_desc0 + ((b * 2048) >> 4);
 #pragma unroll
-            for (int limb = 0; limb < 2; ++limb) {
+            for (int k = 0; k < 4; ++k) {             // 32 tokens per step = 4 atoms of 8 tokens
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {           // 32 tokens per step = 4 atoms of 8 tokens
+              for (int limb = 0; limb < 2; ++limb) {  // the two limb chains alternate
                 const uint64_t ad = vh_desc0 + ((b * Sm::kVhBytes + limb * kTT * 128 + k * 4096) >> 4);
                 umma_i8_ss(d + limb * 16, ad, pb + ((k * 32) >> 4), id_v, k != 0);
               }
             }
             umma_commit(&pv_full[b]);
-            umma_commit(&vh_free[b]);
-            umma_commit(&p_free[b]);
-            ++np;
-            progress = true;
           }
         }
-        if (progress) {
-          last = globaltimer_ns();
-        } else if (globaltimer_ns() - last > 2000000000ull) {
-          fail();
-          break;
-        }
       }
+      if (!ok && !*abort_s) fail();
+      // Every MMA this thread issued completes before TMEM is released.
+      umma_commit(&drain[warp == 1 ? 0 : 1]);
+      mbar_wait(&drain[warp == 1 ? 0 : 1], 0);
     }
   } else if (warp < 6) {
     // ------------------------------------------------- key operands (TMEM)
@@ -495,14 +494,54 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
       }
     }
   } else if (warp < 10) {
-    // ------------------------------------------------ value operands (smem)
-    const int row = tid - 192;                    // token within the tile
+    // ------------------------------- value operands (smem), value epilogue
+    const int row = tid - 192;                    // token within the tile (operands)
+    const int q = warp & 3;                       // lane quadrant (warps 6..9 -> 2,3,0,1)
+    const int crd = q * 32 + lane;                // coordinate = TMEM lane (epilogue)
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t v1t[2] = {tab[12], tab[13]}, v2t[2] = {tab[16], tab[17]};
     int j = 0;
     bool stop = false;
+    float acc[2][kRowsTc];                        // even / odd tiles of the item
+    // Value epilogue of tile jj (this thread = coordinate crd): wait for its
+    // PV product, then for ring slot jj % 4 to carry tag jj (the softmax warps
+    // write the tile's corrections and scale, fence, then the tag; the slot is
+    // rewritten only after PV(jj + 2), which needs this epilogue's do_free).
+    auto value_epilogue = [&](int jj) -> bool {
+      const int b2 = jj & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&pv_full[b2], (jj >> 1) & 1))) return false;
+      tc_fence_after();
+      uint32_t d[32];
+      tmem_ld32(lane_addr + kColDo + b2 * 32, d);
+      volatile int* tag = reinterpret_cast<volatile int*>(ring + (jj & 3) * 8 + 5);
+      bool tag_ok = *tag == jj;
+      if (!tag_ok) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!(tag_ok = (*tag == jj)) && globaltimer_ns() - t0 < 2000000000ull) {
+        }
+      }
+      __threadfence_block();
+      const float4 c4 = reinterpret_cast<const float4*>(ring + (jj & 3) * 8)[0];
+      const float spv = ring[(jj & 3) * 8 + 4] * v_scale;
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&do_free[b2]);
+      if (!__all_sync(0xffffffffu, tag_ok)) return false;
+      const float corr[kRowsTc] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+      for (int r = 0; r < kRowsTc; ++r) {
+        // column (r, weight limb l) = 3 r + l in each value-limb chain
+        const float hi = limb_sum3(d + 3 * r), lo = limb_sum3(d + 16 + 3 * r);
+        acc[b2][r] = fmaf(acc[b2][r], corr[r], spv * fmaf(lo, 1.f / 128.f, hi));
+      }
+      return true;
+    };
     for (int item = blockIdx.x; !stop && item < A.n_items; item += gridDim.x) {
       int64_t tb, te;
       const int nt_tiles = item_tiles(item, tb, te);
+#pragma unroll
+      for (int r = 0; r < kRowsTc; ++r) acc[0][r] = acc[1][r] = 0.f;
       for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
         const int s = j % kStages;
         const int b = j & 1;
@@ -551,16 +590,49 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&vh_full[b]);
+        // Fold the previous tile of this item (its PV product is under way or done).
+        if (tj >= 1 && !value_epilogue(j - 1)) {
+          if (lane == 0) fail();
+          stop = true;
+          break;
+        }
+      }
+      if (stop) break;
+      if (!value_epilogue(j - 1)) {
+        if (lane == 0) fail();
+        break;
+      }
+      // Rotated-value partials of the item's even and odd tiles (records
+      // 2 split + parity; m and l come from the softmax warps).
+      const int64_t unit = item / sh.n_splits;
+      const int split = item % sh.n_splits;
+      const int kv = static_cast<int>(unit % sh.hkv), bb = static_cast<int>(unit / sh.hkv);
+      const int G = sh.hq / sh.hkv;
+#pragma unroll
+      for (int r = 0; r < kRowsTc; ++r) {
+        const int64_t qr = (int64_t(bb) * sh.hq + kv * G + r / sh.nq) * sh.nq + r % sh.nq;
+        float* pr = a.part + (qr * sh.n_parts + 2 * split) * (kD + 2) + crd;
+        pr[0] = acc[0][r];
+        pr[kD + 2] = acc[1][r];
       }
     }
-  } else {
-    // ------------------------------------- scores, softmax, value epilogue
-    const int cw = warp - 10;                     // 0..3
-    const int q = warp & 3;                       // lane quadrant (warps 10..13 -> 2,3,0,1)
-    const int lrow = q * 32 + lane;               // TMEM lane = token / coordinate
+  } else if (warp < 14) {
+    // ------------------- scores and softmax: even and odd tiles kept apart
+    constexpr int wg = 0;
+    const int cw = warp - 10;                     // warp within the group
+    const int q = warp & 3;                       // lane quadrant (2,3,0,1 per group)
+    const int lrow = q * 32 + lane;               // TMEM lane = token
+    const int bar_id = 1 + wg;
+    float* gred = red + wg * 64;
+    float* gred2 = red2 + wg * 16;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const float alpha = static_cast<float>(dev::kSqrtHalfPi / kD);
     constexpr float kLog2e = 1.4426950408889634f;
+    constexpr float kMagic = 12582912.f;          // 1.5 * 2^23: x + kMagic rounds x to an integer
+    // Byte offsets of this token's column in the 12 used rows of a weight tile.
+    uint32_t poff[12];
+#pragma unroll
+    for (int n = 0; n < 12; ++n) poff[n] = sw_byte(n, lrow);
     int j = 0, item_idx = 0;
     bool stop = false;
     for (int item = blockIdx.x; item < A.n_items && !stop; item += gridDim.x, ++item_idx) {
@@ -575,33 +647,37 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
 #pragma unroll
       for (int r = 0; r < kRowsTc; ++r)
         qrow[r] = (int64_t(bb) * sh.hq + kv * G + r / sh.nq) * sh.nq + r % sh.nq;
-      // ---- item prologue: row scales, the item's largest ||v||, B tiles.
+      // ---- item prologue: row scales, the item's largest ||v||; group 0
+      // also writes the item's B tiles.
       const int ib = item_idx & 1;
-      float qv[kRowsTc], sv[kRowsTc];
-      float sq[kRowsTc], ss[kRowsTc], ssum[kRowsTc];
+      float sq[kRowsTc], ss[kRowsTc], ssum[kRowsTc], sp;
       {
-        const float jscale = __uint_as_float(static_cast<uint32_t>(127 - (lrow & 7)) << 23);   // 2^-(i mod 8)
-        float loc[12];
+        const int crd = lrow;                     // thread = coordinate here
+        const float jscale = __uint_as_float(static_cast<uint32_t>(127 - (crd & 7)) << 23);   // 2^-(i mod 8)
+        float qv[kRowsTc], sv[kRowsTc], loc[13];
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          qv[r] = a.qs[qrow[r] * 2 * kD + lrow];
-          sv[r] = a.qs[qrow[r] * 2 * kD + kD + lrow];
+          qv[r] = a.qs[qrow[r] * 2 * kD + crd];
+          sv[r] = a.qs[qrow[r] * 2 * kD + kD + crd];
           loc[r] = fabsf(qv[r]);
           loc[4 + r] = fabsf(sv[r]) * jscale;
           loc[8 + r] = sv[r];
         }
+        float vm = 0.f;
+        for (int64_t t = tb + lrow; t < te; t += kTT) vm = fmaxf(vm, __ldg(a.vnorm + row0 + t));
+        loc[12] = vm;
 #pragma unroll
-        for (int u = 0; u < 12; ++u) {
+        for (int u = 0; u < 13; ++u) {
           const float x = (u >= 8 && u < 12) ? warp_sum(loc[u]) : warp_max(loc[u]);
-          if (lane == 0) red[cw * 16 + u] = x;
+          if (lane == 0) gred[cw * 16 + u] = x;
         }
-        wg_sync(1);
-        float tot[12];
+        wg_sync(bar_id);
+        float tot[13];
 #pragma unroll
-        for (int u = 0; u < 12; ++u) {
-          float x = red[u];
+        for (int u = 0; u < 13; ++u) {
+          float x = gred[u];
 #pragma unroll
-          for (int w2 = 1; w2 < 4; ++w2) x = (u >= 8 && u < 12) ? x + red[w2 * 16 + u] : fmaxf(x, red[w2 * 16 + u]);
+          for (int w2 = 1; w2 < 4; ++w2) x = (u >= 8 && u < 12) ? x + gred[w2 * 16 + u] : fmaxf(x, gred[w2 * 16 + u]);
           tot[u] = x;
         }
 #pragma unroll
@@ -610,76 +686,63 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
           ss[r] = tot[4 + r] > 0.f ? tot[4 + r] / 127.f : 1.f;
           ssum[r] = tot[8 + r];
         }
-        // B tiles: B1/B2/B3 rows 4 r + w hold limb w, w-1, w-2 of q_rot row r;
-        // Bs rows 4 r + l hold limb l of s' at K position 16 (i mod 8) + i / 8.
-        unsigned char* bt = sm + Sm::kOffB + ib * 4 * 2048;
-        const int ks = 16 * (lrow & 7) + (lrow >> 3);
+        // Weights p ||v|| <= max ||v|| of the item (p <= 1): three int8 limbs.
+        sp = tot[12] > 0.f ? tot[12] / 127.f : 1.f;
+        if (wg == 0) {
+          // B tiles: B1/B2/B3 rows 4 r + w hold limb w, w-1, w-2 of q_rot row r;
+          // Bs rows 4 r + l hold limb l of s' at K position 16 (i mod 8) + i / 8.
+          unsigned char* bt = sm + Sm::kOffB + ib * 4 * 2048;
+          const int ks = 16 * (crd & 7) + (crd >> 3);
 #pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          int lq[4], ls[4];
-          limbs4(qv[r] / sq[r], lq);
-          limbs4(sv[r] * jscale / ss[r], ls);
+          for (int r = 0; r < kRowsTc; ++r) {
+            int lq[4], ls[4];
+            limbs4(qv[r] / sq[r], lq);
+            limbs4(sv[r] * jscale / ss[r], ls);
 #pragma unroll
-          for (int w2 = 0; w2 < 4; ++w2) {
-            bt[sw_byte(4 * r + w2, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(lq[w2]));
-            bt[2048 + sw_byte(4 * r + w2, lrow)] =
-                static_cast<unsigned char>(static_cast<int8_t>(w2 >= 1 ? lq[w2 - 1] : 0));
-            bt[4096 + sw_byte(4 * r + w2, lrow)] =
-                static_cast<unsigned char>(static_cast<int8_t>(w2 >= 2 ? lq[w2 - 2] : 0));
-            bt[6144 + sw_byte(4 * r + w2, ks)] = static_cast<unsigned char>(static_cast<int8_t>(ls[w2]));
+            for (int w2 = 0; w2 < 4; ++w2) {
+              bt[sw_byte(4 * r + w2, crd)] = static_cast<unsigned char>(static_cast<int8_t>(lq[w2]));
+              bt[2048 + sw_byte(4 * r + w2, crd)] =
+                  static_cast<unsigned char>(static_cast<int8_t>(w2 >= 1 ? lq[w2 - 1] : 0));
+              bt[4096 + sw_byte(4 * r + w2, crd)] =
+                  static_cast<unsigned char>(static_cast<int8_t>(w2 >= 2 ? lq[w2 - 2] : 0));
+              bt[6144 + sw_byte(4 * r + w2, ks)] = static_cast<unsigned char>(static_cast<int8_t>(ls[w2]));
+            }
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&b_full[ib]);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&b_full[ib]);
       }
+      const float inv_sp = 1.f / sp;
       float kq[kRowsTc], ks2[kRowsTc];
+      const float kr = a.scale * alpha;
 #pragma unroll
       for (int r = 0; r < kRowsTc; ++r) {
         kq[r] = a.scale * k_scale * sq[r];
         ks2[r] = 2.f * ss[r];
       }
-      float m_run[kRowsTc], l_part[kRowsTc], acc[kRowsTc];
-      float corr_prev[kRowsTc], sp_prev[kRowsTc];       // of the tile whose values fold next
+      // Running maximum and sum of the item's even and odd tiles, kept apart:
+      // the value warps accumulate the two parities separately and each
+      // leaves its own partial record.
+      // m_run / l_part: state of the parity of the tile being processed;
+      // m_oth / l_oth: the other parity's (swapped after every tile).
+      float m_run[kRowsTc], l_part[kRowsTc], m_oth[kRowsTc], l_oth[kRowsTc];
 #pragma unroll
       for (int r = 0; r < kRowsTc; ++r) {
-        m_run[r] = -INFINITY;
-        l_part[r] = 0.f;
-        acc[r] = 0.f;
-        corr_prev[r] = 0.f;
-        sp_prev[r] = 1.f;
+        m_run[r] = m_oth[r] = -INFINITY;
+        l_part[r] = l_oth[r] = 0.f;
       }
-      // Value epilogue of tile jj (this thread = coordinate lrow).
-      auto value_epilogue = [&](int jj) -> bool {
-        const int b2 = jj & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_full[b2], (jj >> 1) & 1))) return false;
-        tc_fence_after();
-        uint32_t d[32];
-        tmem_ld32(lane_addr + kColDo + b2 * 32, d);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&do_free[b2]);
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          // column (r, weight limb) = 2 r + limb in each value-limb chain
-          const float hi = fmaf(static_cast<float>(static_cast<int>(d[2 * r + 1])), 1.f / 128.f,
-                                static_cast<float>(static_cast<int>(d[2 * r])));
-          const float lo = fmaf(static_cast<float>(static_cast<int>(d[16 + 2 * r + 1])), 1.f / 128.f,
-                                static_cast<float>(static_cast<int>(d[16 + 2 * r])));
-          acc[r] = fmaf(acc[r], corr_prev[r], v_scale * sp_prev[r] * fmaf(lo, 1.f / 128.f, hi));
-        }
-        return true;
-      };
-      // Norms of the next tile are loaded one tile ahead.
+      const int j0 = j;
+      // Norms are loaded one tile ahead.
       float kn_n = 0.f, rn_n = 0.f, vn_n = 0.f;
       if (lrow < te - tb) {
         kn_n = __ldg(a.knorm + row0 + tb + lrow);
         rn_n = __ldg(a.krnorm + row0 + tb + lrow);
         vn_n = __ldg(a.vnorm + row0 + tb + lrow);
       }
-      for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
-        const int b = j & 1;
+      for (int tj = 0; tj < nt_tiles; ++tj) {
+        const int jt = j0 + tj;
+        const int b = jt & 1;
         const int64_t t0 = tb + int64_t(tj) * kTT;
         const int nt = static_cast<int>((te - t0 < kTT) ? te - t0 : kTT);
         const bool valid = lrow < nt;
@@ -689,7 +752,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
           rn_n = __ldg(a.krnorm + row0 + t0 + kTT + lrow);
           vn_n = __ldg(a.vnorm + row0 + t0 + kTT + lrow);
         }
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (jt >> 1) & 1));
         tc_fence_after();
         uint32_t d[32];
         tmem_ld32(lane_addr + kColDs + b * 32, d);
@@ -701,33 +764,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         bool need = false;
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          const float mse = limb_sum4(d + 4 * r);
+          // weights 0, 1, 2 of the key limb products (weight 3 is below 1e-6)
+          const float mse = limb_sum3(d + 4 * r);
           const float sgn = limb_sum4(d + 16 + 4 * r);
           const float qjl = fmaf(ks2[r], sgn, -ssum[r]);
-          score[r] = valid ? fmaf(kq[r] * kn, mse, a.scale * alpha * rn * qjl) : -INFINITY;
+          score[r] = valid ? fmaf(kq[r] * kn, mse, kr * rn * qjl) : -INFINITY;
           need |= score[r] > m_run[r];
         }
         if (a.scores_out && valid) {
 #pragma unroll
           for (int r = 0; r < kRowsTc; ++r) a.scores_out[qrow[r] * sh.n_ctx + t0 + lrow] = score[r];
         }
-        // Per-warp maxima of z = score log2 e + log2 ||v|| (the largest weight
-        // p ||v|| of the tile, up to the running maximum), published before the
-        // vote barrier; slots alternate by tile parity.
-        {
-          const float lv = valid ? __log2f(vn) : -INFINITY;
-#pragma unroll
-          for (int r = 0; r < kRowsTc; ++r) {
-            const float zm = warp_max(valid ? fmaf(score[r], kLog2e, lv) : -INFINITY);
-            if (lane == 0) zred[(b * 4 + cw) * 4 + r] = zm;
-          }
-        }
         float corr[kRowsTc];
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) corr[r] = 1.f;
         // The running maximum moves only when some score of the tile exceeds it.
-        if (wg_sync_or(1, need || !ok || *abort_s != 0)) {
-          if (wg_sync_or(1, !ok || *abort_s != 0)) {
+        if (wg_sync_or(bar_id, need || !ok || *abort_s != 0)) {
+          if (wg_sync_or(bar_id, !ok || *abort_s != 0)) {
             if (!ok && lane == 0 && cw == 0) fail();
             stop = true;
             break;
@@ -735,88 +788,88 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
 #pragma unroll
           for (int r = 0; r < kRowsTc; ++r) {
             const float mx = warp_max(score[r]);
-            if (lane == 0) red[cw * 16 + r] = mx;
+            if (lane == 0) gred[cw * 16 + r] = mx;
           }
-          wg_sync(1);
+          wg_sync(bar_id);
 #pragma unroll
           for (int r = 0; r < kRowsTc; ++r) {
-            float mx = red[r];
+            float mx = gred[r];
 #pragma unroll
-            for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, red[w2 * 16 + r]);
+            for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, gred[w2 * 16 + r]);
             const float m_new = fmaxf(m_run[r], mx);
-            corr[r] = (m_run[r] == -INFINITY) ? 0.f : exp2f((m_run[r] - m_new) * kLog2e);
+            corr[r] = (m_run[r] == -INFINITY) ? 0.f : ex2((m_run[r] - m_new) * kLog2e);
             l_part[r] *= corr[r];
             m_run[r] = m_new;
-          }
-        }
-        // Weight scale of each row: max_t p ||v|| / 127, with a margin so the
-        // largest limb stays at or below 127 after rounding.
-        float inv_sp[kRowsTc], sp_cur[kRowsTc];
-        {
-          const float4* zr = reinterpret_cast<const float4*>(zred + b * 16);
-          const float4 z0 = zr[0], z1 = zr[1], z2 = zr[2], z3 = zr[3];
-          const float zmax[kRowsTc] = {fmaxf(fmaxf(z0.x, z1.x), fmaxf(z2.x, z3.x)),
-                                       fmaxf(fmaxf(z0.y, z1.y), fmaxf(z2.y, z3.y)),
-                                       fmaxf(fmaxf(z0.z, z1.z), fmaxf(z2.z, z3.z)),
-                                       fmaxf(fmaxf(z0.w, z1.w), fmaxf(z2.w, z3.w))};
-#pragma unroll
-          for (int r = 0; r < kRowsTc; ++r) {
-            float wmax = exp2f(zmax[r] - m_run[r] * kLog2e) * (1.f + 1.f / 4096.f);
-            if (!(wmax > 0.f)) wmax = 127.f;           // no weight in this tile (all ||v|| = 0)
-            sp_cur[r] = wmax * (1.f / 127.f);
-            inv_sp[r] = 127.f / wmax;
           }
         }
         float p[kRowsTc];
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          p[r] = valid ? exp2f((score[r] - m_run[r]) * kLog2e) : 0.f;
+          p[r] = valid ? ex2((score[r] - m_run[r]) * kLog2e) : 0.f;
           l_part[r] += p[r];
         }
-        // Weight limbs into the P tile (row 2 r + limb, column = token).
-        if (!__all_sync(0xffffffffu, mbar_wait(&p_free[b], ((j >> 1) & 1) ^ 1)) && lane == 0) fail();
+        // Weight limbs into the P tile (row 3 r + limb, column = token); the
+        // tile's corrections and scale go to ring[jt % 4] for the value warps.
+        if (!__all_sync(0xffffffffu, mbar_wait(&p_free[b], ((jt >> 1) & 1) ^ 1)) && lane == 0) fail();
+        if (lrow == 0) {
+          float* slot = ring + (jt & 3) * 8;
+          reinterpret_cast<float4*>(slot)[0] = make_float4(corr[0], corr[1], corr[2], corr[3]);
+          slot[4] = sp;
+          __threadfence_block();
+          *reinterpret_cast<volatile int*>(slot + 5) = jt;
+        }
         unsigned char* pt = sm + Sm::kOffP + b * 2048;
+        const float wv = vn * inv_sp;
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          const float x = fminf(p[r] * vn * inv_sp[r], 127.f);
-          const int l0 = __float2int_rn(x);
-          const int l1 = __float2int_rn((x - static_cast<float>(l0)) * 128.f);
-          pt[sw_byte(2 * r, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l0));
-          pt[sw_byte(2 * r + 1, lrow)] = static_cast<unsigned char>(static_cast<int8_t>(l1));
+          float x = fminf(p[r] * wv, 127.f);
+#pragma unroll
+          for (int l = 0; l < 3; ++l) {
+            const float t = x + kMagic;                   // rint(x) in the low mantissa bits
+            pt[poff[3 * r + l]] = static_cast<unsigned char>(__float_as_uint(t));
+            x = (x - (t - kMagic)) * 128.f;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
-        // Fold the previous tile's values (its correction comes first).
-        if (tj >= 1 && !value_epilogue(j - 1)) {
-          if (lane == 0) fail();
-        }
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          corr_prev[r] = corr[r];
-          sp_prev[r] = sp_cur[r];
+          const float tm = m_run[r], tl = l_part[r];
+          m_run[r] = m_oth[r];
+          l_part[r] = l_oth[r];
+          m_oth[r] = tm;
+          l_oth[r] = tl;
         }
       }
+      j = j0 + nt_tiles;
       if (stop) break;
-      // Last tile of the item, then the partials.
-      if (!value_epilogue(j - 1) && lane == 0) fail();
-      float lsum[kRowsTc];
+      // Softmax statistics of the two partials (the value warps write acc).
+      // m_run / l_part now hold the parity of tile j0 + nt_tiles, m_oth / l_oth
+      // the other one.
+      const int par_run = (j0 + nt_tiles) & 1;
 #pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) {
-        const float x = warp_sum(l_part[r]);
-        if (lane == 0) red2[cw * 4 + r] = x;
-      }
-      wg_sync(1);
+      for (int par = 0; par < 2; ++par) {
+        const bool use_run = par == par_run;
+        float lsum[kRowsTc];
 #pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) lsum[r] = red2[r] + red2[4 + r] + red2[8 + r] + red2[12 + r];
-      const int64_t pbase = (int64_t(split)) * (kD + 2);
+        for (int r = 0; r < kRowsTc; ++r) {
+          const float x = warp_sum(use_run ? l_part[r] : l_oth[r]);
+          if (lane == 0) gred2[cw * 4 + r] = x;
+        }
+        wg_sync(bar_id);
 #pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) {
-        float* pr = a.part + qrow[r] * sh.n_splits * (kD + 2) + pbase;
-        pr[lrow] = acc[r];
+        for (int r = 0; r < kRowsTc; ++r) lsum[r] = gred2[r] + gred2[4 + r] + gred2[8 + r] + gred2[12 + r];
+        wg_sync(bar_id);
         if (lrow == 0) {
-          pr[kD] = m_run[r];
-          pr[kD + 1] = lsum[r];
+          // record 2 split + parity of the tiles' index j
+          const int rec = 2 * split + par;
+#pragma unroll
+          for (int r = 0; r < kRowsTc; ++r) {
+            float* pr = a.part + (qrow[r] * sh.n_parts + rec) * (kD + 2);
+            pr[kD] = use_run ? m_run[r] : m_oth[r];
+            pr[kD + 1] = lsum[r];
+          }
         }
       }
     }
@@ -828,10 +881,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    if (lane == 0) {
-      umma_commit(drain);
-      mbar_wait(drain, 0);
-    }
     __syncwarp();
     tmem_dealloc(tmem, kTmemColsTc);
   }

@@ -15,6 +15,7 @@ struct DecodeShape {
   int rows_per_cta;   // R
   int row_blocks;     // (hq/hkv*nq) / R
   int n_splits;
+  int n_parts;        // partial records per query row: n_splits, or 2 n_splits (tensor-core path)
   int64_t chunk;      // tokens per split (multiple of kT)
   int64_t n_rows;     // batch*hq*nq
 };
@@ -42,7 +43,7 @@ struct DecodeArgs {
   int out_dtype;
   float* scores_out;
   float* qs;     // [n_rows][2][d]  q_rot then s
-  float* part;   // [n_rows][n_splits][d + 2]  acc..., m, l
+  float* part;   // [n_rows][n_parts][d + 2]  acc..., m, l
   int32_t* d_status;
 };
 

@@ -335,10 +335,10 @@ __global__ void __launch_bounds__(kT2) decode_main_v2(DecodeArgs a) {
     float sum = 0.f;
 #pragma unroll
     for (int u = 0; u < kSub; ++u) sum += part[(u * D + i) * R + r];
-    a.part[(qrow(r) * sh.n_splits + split) * (D + 2) + i] = sum;
+    a.part[(qrow(r) * sh.n_parts + split) * (D + 2) + i] = sum;
   }
   if (tid < R) {
-    float* p = a.part + (qrow(tid) * sh.n_splits + split) * (D + 2);
+    float* p = a.part + (qrow(tid) * sh.n_parts + split) * (D + 2);
     p[D] = s_m[tid];
     p[D + 1] = s_l[tid];
   }

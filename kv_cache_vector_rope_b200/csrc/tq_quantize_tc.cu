@@ -386,9 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         }
         if (progress) {
           last = globaltimer_ns();
-        } else if (globaltimer_ns() - last > 2000000000ull) {
-          fail();
-          break;
+        } else {
+          __nanosleep(32);              // nothing ready: leave the issue slots to the other warps
+          if (globaltimer_ns() - last > 2000000000ull) {
+            fail();
+            break;
+          }
         }
       }
     }
