@@ -12,8 +12,10 @@ value = context tokens per second: every step quantises all 32x8 key and value
 vectors of each of the batch x 32768 positions and scores them against the 32
 query heads of every layer (tokens per step = batch x context).
 Per-phase figures (quantize tokens/s, decode keys scored/s, HBM GB/s) sit in
-"phases"; "roofline" describes the dominant kernel (quantize) and
-"roofline_decode" the decode path.
+"phases". "roofline" describes the dominant call of the step, tq_quantize_kv of
+one layer's keys, from CUDA events around every such call in the timed region;
+"roofline_value" and "roofline_decode" do the same for the value quantisation
+and the decode call of a layer.
 
 Timing: W untimed warm-up steps, then K steps between CUDA events on the
 launching stream, bracketed by barrier + synchronize; max over ranks. Inputs
@@ -43,6 +45,11 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "decode-attn keys scored/s & HBM GB/s on 3+1-bit KV; quantize tokens/s"
+# DRAM bytes (read + write) per call from the ncu captures summarised under
+# profiles/ (context-8192 case, scaled x4 to the 32768-token call; traffic grows
+# with the vectors processed). None until measured for the current kernels.
+NCU_TRAFFIC = {"quantize_key": None, "quantize_value": None, "decode": None}
+
 WORKLOAD = ("Llama-3.1-8B-shaped decode: 32 layers, batch 8, 32 q / 8 kv heads, head_dim 128, context 32768, "
             "bf16 N(0,1) K/V with 2% channels x10; 3-bit+QJL keys, 3-bit values")
 
@@ -233,31 +240,31 @@ def run_ours(args, world, rank):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def quantize_layer(l, ev=None):
-        tq.tq_quantize_kv(lay, True, K[l], kp[l], Pi, cd, td, S=S, d_status=status)
-        tq.tq_quantize_kv(lay, False, V[l], vp[l], Pi, cd, td, d_status=status)
-
-    def decode_layer(l):
-        tq.tq_decode_attention(lay, Q[l], kp[l], vp[l], HKV, N, Pi, Pi, S, cd, cd, out[l], ws, d_status=status)
-
-    def step(rec=None):
-        if rec is not None:
-            rec[0].record(stream)
+    def step(ev=None):
+        # ev: events [K start, K end = V start, V end] per layer, then decode
+        # boundaries (L + 1), all on the launching stream.
         for l in range(L):
-            quantize_layer(l)
-        if rec is not None:
-            rec[1].record(stream)
+            if ev is not None:
+                ev[3 * l].record(stream)
+            tq.tq_quantize_kv(lay, True, K[l], kp[l], Pi, cd, td, S=S, d_status=status)
+            if ev is not None:
+                ev[3 * l + 1].record(stream)
+            tq.tq_quantize_kv(lay, False, V[l], vp[l], Pi, cd, td, d_status=status)
+            if ev is not None:
+                ev[3 * l + 2].record(stream)
         for l in range(L):
-            decode_layer(l)
-        if rec is not None:
-            rec[2].record(stream)
+            if ev is not None:
+                ev[3 * L + l].record(stream)
+            tq.tq_decode_attention(lay, Q[l], kp[l], vp[l], HKV, N, Pi, Pi, S, cd, cd, out[l], ws, d_status=status)
+        if ev is not None:
+            ev[4 * L].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert int(status.item()) == 0, f"device status {int(status.item())}"
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * L + 1)] for _ in range(args.steps)]
     clocks = ClockSampler(dev.index)
     barrier(world)
     torch.cuda.synchronize()
@@ -270,9 +277,14 @@ def run_ours(args, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
     total_ms = start.elapsed_time(end)
-    q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    d_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    n_calls = args.steps * L
+    k_ms = sum(e[3 * l].elapsed_time(e[3 * l + 1]) for e in ev for l in range(L)) / n_calls
+    v_ms = sum(e[3 * l + 1].elapsed_time(e[3 * l + 2]) for e in ev for l in range(L)) / n_calls
+    dl_ms = sum(e[3 * L + l].elapsed_time(e[3 * L + l + 1]) for e in ev for l in range(L)) / n_calls
+    q_ms = sum(e[0].elapsed_time(e[3 * L - 1]) for e in ev) / args.steps
+    d_ms = sum(e[3 * L].elapsed_time(e[4 * L]) for e in ev) / args.steps
     total_ms = max_over_ranks(world, total_ms)
     ms_step = total_ms / args.steps
 
@@ -293,6 +305,16 @@ def run_ours(args, world, rank):
     q_gbs = quant_bytes_step / (q_ms * 1e-3) / 1e9
     d_gbs = dec_bytes_step / (d_ms * 1e-3) / 1e9
     value = world * tokens_step / (ms_step * 1e-3)
+    # Per-call rooflines (CUDA events around each call on the launching stream).
+    k_call_gbs = n_vec * k_bytes / (k_ms * 1e-3) / 1e9
+    v_call_gbs = n_vec * v_bytes / (v_ms * 1e-3) / 1e9
+    d_call_gbs = n_vec * (48 + 16 + 4 + 4 + 48 + 4) / (dl_ms * 1e-3) / 1e9
+    full = (N == 32768 and L == shape.layers)
+
+    def roof(kernel, achieved, per_unit, traffic_key):
+        return {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": NCU_TRAFFIC.get(traffic_key) if full else None,
+                "peak_source": peak_src, "per_unit": per_unit}
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -305,17 +327,22 @@ def run_ours(args, world, rank):
                    "parallelism": f"replicas x{world} (independent caches, no collective)"},
         "phases": {
             "quantize": {"ms": q_ms, "tokens_per_s": tokens_step / (q_ms * 1e-3),
-                         "token_heads_per_s": 2 * L * n_vec / (q_ms * 1e-3), "algorithmic_gbs": q_gbs},
-            "decode": {"ms": d_ms, "keys_scored_per_s": keys_scored_step / (d_ms * 1e-3), "algorithmic_gbs": d_gbs},
+                         "token_heads_per_s": 2 * L * n_vec / (q_ms * 1e-3), "algorithmic_gbs": q_gbs,
+                         "key_call_us": 1e3 * k_ms, "value_call_us": 1e3 * v_ms},
+            "decode": {"ms": d_ms, "keys_scored_per_s": keys_scored_step / (d_ms * 1e-3), "algorithmic_gbs": d_gbs,
+                       "call_us": 1e3 * dl_ms},
         },
-        "roofline": {"kernel": "quantize_kernel", "bound": "hbm", "achieved": q_gbs, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": q_gbs / hbm_peak, "traffic": None, "peak_source": peak_src,
-                     "per_unit": "bf16 in 256 B + packed out 72 B (key) / 52 B (value) per vector"},
-        "roofline_decode": {"kernel": "decode_main (+prologue, combine)", "bound": "hbm", "achieved": d_gbs,
-                            "peak": hbm_peak, "unit": "GB/s", "frac": d_gbs / hbm_peak, "traffic": None,
-                            "peak_source": peak_src, "per_unit": "124 B per (token, kv head)"},
+        # The dominant call of the step: tq_quantize_kv of one layer's keys
+        # (quantize_tc_kernel<128, key, 3> + quantize_fixup), 2,097,152 vectors.
+        "roofline": roof("tq_quantize_kv(keys): quantize_tc_kernel<128,key,3> + quantize_fixup", k_call_gbs,
+                         "bf16 in 256 B + packed out 72 B per key vector; 2,097,152 vectors per call", "quantize_key"),
+        "roofline_value": roof("tq_quantize_kv(values): quantize_tc_kernel<128,value,3> + quantize_fixup",
+                               v_call_gbs, "bf16 in 256 B + packed out 52 B per value vector", "quantize_value"),
+        "roofline_decode": roof("tq_decode_attention: decode_prologue + decode_tc_kernel<3> + decode_combine",
+                                d_call_gbs, "124 B per (token, kv head); 2,097,152 per call", "decode"),
         "clocks": clk,
-        "gpu_launches": args.steps * L * (2 + 3),
+        # kernels per layer: 2 (key quantize + fixup) + 2 (values) + 3 (decode)
+        "gpu_launches": args.steps * L * 7,
     }
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, tq, lay, K, V, Q, kp, vp, out, ws, Pi, S, cd, td, status, shape, world)

@@ -95,6 +95,7 @@ __device__ __forceinline__ void row_coords(const DecodeShape& s, int64_t row, in
 // ---------------------------------------------------------------------------
 constexpr int kBlkRows = 16;
 constexpr int kBlkThreads = 256;
+constexpr int kCombChunk = 64;       // partial records whose weights are staged at a time
 
 struct RowBlocks {
   int rows_per_group, blocks_per_group, n_blocks;
@@ -112,12 +113,32 @@ RowBlocks row_blocks(const DecodeShape& s, int64_t pi_stride) {
 inline int row_groups(int d) { return d <= 64 ? 4 : (d <= 128 ? 2 : 1); }
 inline size_t blk_smem_bytes(int d) { return sizeof(float) * (size_t(d) * (d + 1) + 2 * size_t(d) * kBlkRows); }
 
-// Stages the d x d row-major matrix M into Ms (pitch d+1): warp w copies rows
-// w, w+8, ...; lane l reads columns l, l+32, ... (coalesced).
+// Stages the d x d row-major matrix M into Ms (pitch d+1): every thread first
+// loads its float4s of the matrix (independent, coalesced loads), then stores
+// them.
 __device__ __forceinline__ void stage_matrix(float* Ms, const float* __restrict__ M, int d) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = warp; i < d; i += kBlkThreads / 32)
-    for (int j = lane; j < d; j += 32) Ms[i * (d + 1) + j] = __ldg(M + int64_t(i) * d + j);
+  const int n4 = d * d / 4, q4 = d / 4;
+  constexpr int kMaxPer = (256 * 256 / 4) / kBlkThreads;
+  float4 v[8];
+  for (int e0 = 0; e0 < n4; e0 += 8 * kBlkThreads) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + threadIdx.x + u * kBlkThreads;
+      if (e < n4) v[u] = __ldg(reinterpret_cast<const float4*>(M) + e);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + threadIdx.x + u * kBlkThreads;
+      if (e < n4) {
+        float* dst = Ms + (e / q4) * (d + 1) + 4 * (e % q4);
+        dst[0] = v[u].x;
+        dst[1] = v[u].y;
+        dst[2] = v[u].z;
+        dst[3] = v[u].w;
+      }
+    }
+  }
+  (void)kMaxPer;
 }
 
 // out[r][i] = sum_j Ms[i][j] xs[j][r] (TRANS = false) or sum_j Ms[j][i] xs[j][r]
@@ -423,26 +444,47 @@ __global__ void __launch_bounds__(kBlkThreads) decode_combine(DecodeArgs a, RowB
   const int d = s.d, ns = s.n_parts;
   float* Ms = blk_smem;                       // [d][d+1] Pi_V
   float* os = Ms + d * (d + 1);               // [d][16] merged rotated outputs
-  float* wl = os + d * kBlkRows;              // [16] 1 / L per row; [16] max per row
+  float* wl = os + d * kBlkRows;              // [16] 1 / L per row; [16] max per row; [16][64] weights
   const int g = blockIdx.x / rb.blocks_per_group, sub = blockIdx.x % rb.blocks_per_group;
   const int64_t row0 = int64_t(g) * rb.rows_per_group + sub * kBlkRows;
   const int cnt = min(kBlkRows, rb.rows_per_group - sub * kBlkRows);
   const int kv = a.pi_stride ? g % s.hkv : 0;
   stage_matrix(Ms, a.PiV + kv * a.pi_stride, d);
-  // Row maxima and softmax denominators: warp w handles rows w and w + 8.
+  float* wk = wl + 2 * kBlkRows;               // [16][kCombChunk] record weights
+  // Row maxima and softmax denominators: warp w handles rows w and w + 8;
+  // with at most kCombChunk records the record weights come out of the same
+  // pass (lane k holds records k and k + 32).
+  const bool one_pass = ns <= kCombChunk;
   {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int r = warp; r < kBlkRows; r += kBlkThreads / 32) {
       float M = -INFINITY, L = 0.f;
       if (r < cnt) {
         const float* part = a.part + (row0 + r) * ns * (d + 2);
-        for (int k = lane; k < ns; k += 32) M = fmaxf(M, part[k * (d + 2) + d]);
-        M = warp_max(M);
-        for (int k = lane; k < ns; k += 32) {
-          const float mk = part[k * (d + 2) + d];
-          if (mk > -INFINITY) L += __expf(mk - M) * part[k * (d + 2) + d + 1];
+        if (one_pass) {
+          const bool h0 = lane < ns, h1 = lane + 32 < ns;
+          const float m0 = h0 ? part[lane * (d + 2) + d] : -INFINITY;
+          const float l0 = h0 ? part[lane * (d + 2) + d + 1] : 0.f;
+          const float m1 = h1 ? part[(lane + 32) * (d + 2) + d] : -INFINITY;
+          const float l1 = h1 ? part[(lane + 32) * (d + 2) + d + 1] : 0.f;
+          M = warp_max(fmaxf(m0, m1));
+          const float w0 = m0 > -INFINITY ? __expf(m0 - M) : 0.f;
+          const float w1 = m1 > -INFINITY ? __expf(m1 - M) : 0.f;
+          L = warp_sum(w0 * l0 + w1 * l1);
+          wk[r * kCombChunk + lane] = w0;
+          wk[r * kCombChunk + lane + 32] = w1;
+        } else {
+          for (int k = lane; k < ns; k += 32) M = fmaxf(M, part[k * (d + 2) + d]);
+          M = warp_max(M);
+          for (int k = lane; k < ns; k += 32) {
+            const float mk = part[k * (d + 2) + d];
+            if (mk > -INFINITY) L += __expf(mk - M) * part[k * (d + 2) + d + 1];
+          }
+          L = warp_sum(L);
         }
-        L = warp_sum(L);
+      } else if (one_pass) {
+        wk[r * kCombChunk + lane] = 0.f;
+        wk[r * kCombChunk + lane + 32] = 0.f;
       }
       if (lane == 0) {
         wl[r] = (r < cnt && L > 0.f) ? 1.f / L : 0.f;
@@ -451,20 +493,44 @@ __global__ void __launch_bounds__(kBlkThreads) decode_combine(DecodeArgs a, RowB
     }
   }
   __syncthreads();
-  // Merged rotated output o[r][i] = sum_k e^(m_k - M) acc_k[i] / L.
+  // Merged rotated output o[r][i] = sum_k e^(m_k - M) acc_k[i] / L, with the
+  // weights of kCombChunk records at a time staged in shared memory so the
+  // record loads of a thread are independent (and coalesced over i).
+  for (int e = threadIdx.x; e < kBlkRows * d; e += kBlkThreads) os[(e % d) * kBlkRows + e / d] = 0.f;
+  for (int k0 = 0; k0 < ns; k0 += kCombChunk) {
+    const int kn = min(kCombChunk, ns - k0);
+    __syncthreads();
+    if (!one_pass)
+    for (int e = threadIdx.x; e < kBlkRows * kCombChunk; e += kBlkThreads) {
+      const int r = e / kCombChunk, kk = e % kCombChunk;
+      float w = 0.f;
+      if (r < cnt && kk < kn) {
+        const float mk = a.part[((row0 + r) * ns + k0 + kk) * (d + 2) + d];
+        if (mk > -INFINITY) w = __expf(mk - wl[kBlkRows + r]);
+      }
+      wk[e] = w;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kBlkRows * d; e += kBlkThreads) {
+      const int r = e / d, i = e % d;
+      if (r >= cnt) continue;
+      const float* rec = a.part + ((row0 + r) * ns + k0) * (d + 2) + i;
+      const float* w = wk + r * kCombChunk;
+      float o0 = 0.f, o1 = 0.f;
+      int kk = 0;
+#pragma unroll 4
+      for (; kk + 1 < kn; kk += 2) {
+        o0 = fmaf(w[kk], rec[kk * (d + 2)], o0);
+        o1 = fmaf(w[kk + 1], rec[(kk + 1) * (d + 2)], o1);
+      }
+      if (kk < kn) o0 = fmaf(w[kk], rec[kk * (d + 2)], o0);
+      os[i * kBlkRows + r] += o0 + o1;
+    }
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < kBlkRows * d; e += kBlkThreads) {
     const int r = e / d, i = e % d;
-    float o = 0.f;
-    if (r < cnt) {
-      const float* part = a.part + (row0 + r) * ns * (d + 2);
-      const float M = wl[kBlkRows + r];
-      for (int k = 0; k < ns; ++k) {
-        const float mk = part[k * (d + 2) + d];
-        if (mk > -INFINITY) o = fmaf(__expf(mk - M), part[k * (d + 2) + i], o);
-      }
-      o *= wl[r];
-    }
-    os[i * kBlkRows + r] = o;
+    os[i * kBlkRows + r] *= wl[r];
   }
   __syncthreads();
   float acc[RPG];
@@ -485,7 +551,7 @@ __global__ void __launch_bounds__(kBlkThreads) decode_combine(DecodeArgs a, RowB
 template <bool COMBINE>
 cudaError_t launch_blk(const DecodeArgs& a, cudaStream_t st) {
   const RowBlocks rb = row_blocks(a.sh, a.pi_stride);
-  const size_t smem = blk_smem_bytes(a.sh.d) + (COMBINE ? 2 * kBlkRows * sizeof(float) : 0);
+  const size_t smem = blk_smem_bytes(a.sh.d) + (COMBINE ? (2 + kCombChunk) * kBlkRows * sizeof(float) : 0);
   const int rg = row_groups(a.sh.d);
   auto kern = COMBINE ? (rg == 4 ? decode_combine<4> : rg == 2 ? decode_combine<8> : decode_combine<16>)
                       : (rg == 4 ? decode_prologue<4> : rg == 2 ? decode_prologue<8> : decode_prologue<16>);

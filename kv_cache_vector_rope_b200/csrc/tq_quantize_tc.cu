@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 // range of rows into a shared-memory list; if the list is not empty it stages
 // Pi (and S) in shared memory and its warps take list entries one at a time.
 // ---------------------------------------------------------------------------
-constexpr int kFixThreads = 1024;
+constexpr int kFixThreads = 512;       // 16 warps, 128 registers
 constexpr int kFixList = 16384;      // rows scanned per round (list capacity)
 
 template <int D, bool KEY, int BITS>
@@ -681,8 +681,20 @@ __global__ void __launch_bounds__(kFixThreads, 1) quantize_fixup(TcArgs a) {
       taken = 0;
     }
     __syncthreads();
-    for (int64_t row = w0 + threadIdx.x; row < w1; row += blockDim.x)
-      if (__float_as_uint(flagp[row]) >> 31) list[atomicAdd(&cnt, 1)] = static_cast<int>(row - w0);
+    // Scan: every thread loads its flag words of the window first
+    // (independent loads), then records the flagged rows.
+    {
+      constexpr int kPer = kFixList / kFixThreads;       // rows per thread per window
+      uint32_t fw[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int64_t row = w0 + threadIdx.x + int64_t(u) * kFixThreads;
+        fw[u] = row < w1 ? __float_as_uint(__ldg(flagp + row)) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u)
+        if (fw[u] >> 31) list[atomicAdd(&cnt, 1)] = static_cast<int>(threadIdx.x + u * kFixThreads);
+    }
     __syncthreads();
     const int total = cnt;
     if (total == 0) continue;
