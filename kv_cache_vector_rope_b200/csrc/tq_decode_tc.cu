@@ -146,16 +146,18 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
 
 // 8 three-bit codes (bits 0..23 of x; bits above ignored) -> one word of
 // eight nibbles c0..c7; PRMT reads the low 16 bits as the selector of c0..c3.
+// Each step moves the upper half of every field up by adding a multiple of
+// it (no field carries into the next).
 __device__ __forceinline__ uint32_t nibbles3(uint32_t x) {
-  const uint32_t y = (x & 0xFFFu) | ((x << 4) & 0x0FFF0000u);          // c0-3 | c4-7 in halves
-  const uint32_t z = (y & 0x003F003Fu) | ((y << 2) & 0x3F003F00u);     // two codes per byte
-  return (z & 0x07070707u) | ((z << 1) & 0x70707070u);                 // one code per nibble
+  const uint32_t y = ((x & 0xFFF000u) << 4) | (x & 0xFFFu);            // c0-3 | c4-7 in halves
+  const uint32_t z = y + 3u * (y & 0x0FC00FC0u);                       // two codes per byte
+  return z + (z & 0x38383838u);                                        // one code per nibble
 }
 // 8 two-bit codes (bits 0..15 of x) -> eight nibbles.
 __device__ __forceinline__ uint32_t nibbles2(uint32_t x) {
-  const uint32_t y = (x & 0xFFu) | ((x << 8) & 0x00FF0000u);
-  const uint32_t z = (y & 0x000F000Fu) | ((y << 4) & 0x0F000F00u);
-  return (z & 0x03030303u) | ((z << 2) & 0x30303030u);
+  const uint32_t y = ((x & 0xFF00u) << 8) | (x & 0xFFu);
+  const uint32_t z = y + 15u * (y & 0x00F000F0u);
+  return z + 3u * (z & 0x0C0C0C0Cu);
 }
 // Byte lookup of four codes in a 16-entry table given as four words (codes
 // 0-3 | 4-7 | 8-11 | 12-15); `nib` holds the four 4-bit codes.

@@ -116,52 +116,6 @@ __device__ __forceinline__ void split3(float v, __nv_bfloat16& a, __nv_bfloat16&
   c = __float2bfloat16_rn(r1 - __bfloat162float(b));
 }
 
-// x[4 lane .. 4 lane + KPL) of a bf16 row (KPL = D/32 elements per lane) in fp64.
-template <int D>
-__device__ __forceinline__ void lane_x(const __nv_bfloat16* __restrict__ xrow, double (&xk)[D / 32]) {
-  const int lane = threadIdx.x & 31;
-  if constexpr (D == 128) {
-    const uint2 v = *reinterpret_cast<const uint2*>(xrow + 4 * lane);
-    xk[0] = __uint_as_float(v.x << 16);
-    xk[1] = __uint_as_float(v.x & 0xffff0000u);
-    xk[2] = __uint_as_float(v.y << 16);
-    xk[3] = __uint_as_float(v.y & 0xffff0000u);
-  } else {
-    const uint32_t v = *reinterpret_cast<const uint32_t*>(xrow + 2 * lane);
-    xk[0] = __uint_as_float(v << 16);
-    xk[1] = __uint_as_float(v & 0xffff0000u);
-  }
-}
-
-// Row i of Pi times the lane's slice of x, in fp64 (no reduction).
-template <int D>
-__device__ __forceinline__ double lane_dot(const float* __restrict__ Pi, int i, const double (&xk)[D / 32]) {
-  const int lane = threadIdx.x & 31;
-  if constexpr (D == 128) {
-    const float4 w = __ldg(reinterpret_cast<const float4*>(Pi + i * D) + lane);
-    return fma(double(w.x), xk[0], fma(double(w.y), xk[1], fma(double(w.z), xk[2], double(w.w) * xk[3])));
-  } else {
-    const float2 w = __ldg(reinterpret_cast<const float2*>(Pi + i * D) + lane);
-    return fma(double(w.x), xk[0], double(w.y) * xk[1]);
-  }
-}
-
-// Sum over lanes of v[m] for every m, returned in lane m (31 exchanges).
-__device__ __forceinline__ double transpose_reduce32(double (&v)[32]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) {
-    const bool up = (lane & s) != 0;
-#pragma unroll
-    for (int i = 0; i < s; ++i) {
-      const double send = up ? v[i] : v[i + s];
-      const double keep = up ? v[i + s] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-    }
-  }
-  return v[0];
-}
-
 // Exact code of y64 (zero vector: u = 0).
 template <int NB>
 __device__ __forceinline__ int exact_code(double y64, double nrm64, const float* bnd) {
@@ -174,31 +128,31 @@ __device__ __forceinline__ int exact_code(double y64, double nrm64, const float*
   return c;
 }
 
-// Code of y against thresholds th[] (strict: ties go to the lower code) and
-// the distance from y to the nearest boundary of its cell.
+// Code of y against thresholds th[] (strict: ties go to the lower code);
+// `near` is set when y lies within `band` of a boundary it was compared with
+// (the boundaries of its cell are among them).
 template <int BITS>
-__device__ __forceinline__ int code_of(float y, const float (&th)[(1 << BITS) - 1], float& dmin) {
-  if (BITS == 3) {
+__device__ __forceinline__ int code_guarded(float y, const float (&th)[(1 << BITS) - 1], float band, bool& near) {
+  if constexpr (BITS == 3) {
     const bool b2 = y > th[3];
     const float tA = b2 ? th[5] : th[1];
     const bool b1 = y > tA;
     const float tB = b2 ? (b1 ? th[6] : th[4]) : (b1 ? th[2] : th[0]);
     const bool b0 = y > tB;
-    dmin = fminf(fabsf(y - th[3]), fminf(fabsf(y - tA), fabsf(y - tB)));
+    near |= (fabsf(y - th[3]) < band) | (fabsf(y - tA) < band) | (fabsf(y - tB) < band);
     return (b2 ? 4 : 0) | (b1 ? 2 : 0) | (b0 ? 1 : 0);
-  } else if (BITS == 2) {
+  } else if constexpr (BITS == 2) {
     const bool b1 = y > th[1];
     const float tA = b1 ? th[2] : th[0];
     const bool b0 = y > tA;
-    dmin = fminf(fabsf(y - th[1]), fabsf(y - tA));
+    near |= (fabsf(y - th[1]) < band) | (fabsf(y - tA) < band);
     return (b1 ? 2 : 0) | (b0 ? 1 : 0);
   } else {
     int c = 0;
-    dmin = INFINITY;
 #pragma unroll
     for (int j = 0; j < (1 << BITS) - 1; ++j) {
       c += (y > th[j]) ? 1 : 0;
-      dmin = fminf(dmin, fabsf(y - th[j]));
+      near |= fabsf(y - th[j]) < band;
     }
     return c;
   }
@@ -413,15 +367,21 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         break;
       }
       tc_fence_after();
-      // Pass 1: ||y||^2 from the accumulator.
+      // The whole accumulator row in registers, one wait for the four loads.
+      // Values: the whole accumulator row in registers (one wait), after
+      // which the slot can take the next Y. Keys: two chunks per wait, and
+      // the row is read again for the codes (fewer registers live).
+      constexpr int kGrp1 = KEY ? (C::kChunks >= 2 ? 2 : 1) : C::kChunks;
+      uint32_t yb[D];
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < C::kChunks; ++ch) {
-        uint32_t yb[32];
-        tmem_ld32(lane_addr + ch * 32, yb);
+      for (int ch0 = 0; ch0 < C::kChunks; ch0 += kGrp1) {
+#pragma unroll
+        for (int u = 0; u < kGrp1; ++u)
+          tmem_ld32(lane_addr + (ch0 + u) * 32, *reinterpret_cast<uint32_t(*)[32]>(yb + (ch0 + u) * 32));
         tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) {
+        for (int k = ch0 * 32; k < (ch0 + kGrp1) * 32; k += 4) {
           const float y0 = __uint_as_float(yb[k]), y1 = __uint_as_float(yb[k + 1]);
           const float y2 = __uint_as_float(yb[k + 2]), y3 = __uint_as_float(yb[k + 3]);
           s0 = fmaf(y0, y0, s0);
@@ -429,6 +389,11 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           s2 = fmaf(y2, y2, s2);
           s3 = fmaf(y3, y3, s3);
         }
+      }
+      if (!KEY) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accfree[wg]);
       }
       const float nrm = sqrtf((s0 + s1) + (s2 + s3));
       const float band = kCodeGuard * nrm;
@@ -444,28 +409,29 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           rscale = __uint_as_float(static_cast<uint32_t>(be) << 23);
         }
       }
-      uint32_t rowflag = 0;                  // any coordinate or sign near its decision
+      bool rowflag = false;                  // any coordinate or sign near its decision
       uint32_t codew[C::kChunks][BITS];
       float rsq = 0.f;
 #pragma unroll
       for (int ch = 0; ch < C::kChunks; ++ch) {
-        uint32_t yb[32];
-        tmem_ld32(lane_addr + ch * 32, yb);
-        tmem_ld_wait();
+        if constexpr (KEY) {
+          constexpr int kGrp = C::kChunks >= 2 ? 2 : 1;
+          if (ch % kGrp == 0) {
+#pragma unroll
+            for (int u = 0; u < kGrp; ++u)
+              tmem_ld32(lane_addr + (ch + u) * 32, *reinterpret_cast<uint32_t(*)[32]>(yb + (ch + u) * 32));
+            tmem_ld_wait();
+          }
+        }
         int code[32];
         float r[32];
-        uint32_t flags = 0;
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float y = __uint_as_float(yb[k]);
-          float dmin;
-          const int c = code_of<BITS>(y, th, dmin);
-          if (dmin < band) flags |= 1u << k;
+          const float y = __uint_as_float(yb[ch * 32 + k]);
+          const int c = code_guarded<BITS>(y, th, band, rowflag);
           code[k] = c;
-          r[k] = fmaf(-nrm, cent_s[c], y);
+          if (KEY) r[k] = fmaf(-nrm, cent_s[c], y);
         }
-        rowflag |= flags;
-        // Pack this chunk's codes (32 codes -> BITS words).
 #pragma unroll
         for (int w = 0; w < BITS; ++w) codew[ch][w] = 0u;
 #pragma unroll
@@ -525,19 +491,25 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         }
         tc_fence_after();
         uint32_t words[C::kChunks];
+        uint32_t pb[D];
 #pragma unroll
         for (int ch = 0; ch < C::kChunks; ++ch) {
-          uint32_t pbits[32];
-          tmem_ld32(lane_addr + ch * 32, pbits);
-          tmem_ld_wait();
-          uint32_t word = 0, flags = 0;
+          constexpr int kGrp = C::kChunks >= 2 ? 2 : 1;        // two chunks per wait
+          if (ch % kGrp == 0) {
+#pragma unroll
+            for (int u = 0; u < kGrp; ++u)
+              tmem_ld32(lane_addr + (ch + u) * 32, *reinterpret_cast<uint32_t(*)[32]>(pb + (ch + u) * 32));
+            tmem_ld_wait();
+          }
+          uint32_t word = 0;
+          bool near = false;
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const float p = __uint_as_float(pbits[k]);
+            const float p = __uint_as_float(pb[ch * 32 + k]);
             word |= (p >= 0.f ? 1u : 0u) << k;
-            if (fabsf(p) < sband) flags |= 1u << k;
+            near |= fabsf(p) < sband;
           }
-          rowflag |= flags;
+          rowflag |= near;
           words[ch] = word;
         }
         tc_fence_before();
@@ -553,10 +525,6 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           }
           a.rnorm[v] = rowflag ? __uint_as_float(__float_as_uint(rn) | 0x80000000u) : rn;
         }
-      } else {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&accfree[wg]);
       }
     }
   }
@@ -578,97 +546,166 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 }
 
 // ---------------------------------------------------------------------------
-// Exact recomputation of flagged rows (fp64, one warp per row). The flag is the
-// sign bit of the row's stored ||r|| (keys) or ||x|| (values); every output of
-// the row is rewritten and the flag cleared. One CTA per SM scans a contiguous
-// range of rows into a shared-memory list; if the list is not empty it stages
-// Pi (and S) in shared memory and its warps take list entries one at a time.
+// Exact recomputation of flagged rows (fp64). The flag is the sign bit of the
+// row's stored ||r|| (keys) or ||x|| (values); every output of the row is
+// rewritten and the flag cleared. One CTA per SM scans a contiguous range of
+// rows into a shared-memory list; if the list is not empty it stages Pi^T (and
+// S^T) in shared memory, fp32, laid out so that lane l reads the G = D/32
+// entries of its output coordinates l, l + 32, ... for one input coordinate
+// with one 16-byte (8-byte for d = 64) load. A warp takes kFixBatch rows at a
+// time: the x (later r) of the rows sit in the warp's fp64 scratch and are
+// read as broadcasts; every converted matrix entry serves all rows of the batch.
 // ---------------------------------------------------------------------------
-constexpr int kFixThreads = 512;       // 16 warps, 128 registers
-constexpr int kFixList = 16384;      // rows scanned per round (list capacity)
+constexpr int kFixThreads = 512;       // 16 warps
+constexpr int kFixWarps = kFixThreads / 32;
+constexpr int kFixList = 8192;         // rows scanned per round (list capacity)
+constexpr int kFixBatch = 4;           // rows per warp at a time
 
-template <int D, bool KEY, int BITS>
-__device__ __noinline__ void fix_row(const TcArgs& a, int64_t v, const float* Pis, const float* Ss, const float* cent,
-                                     const float* bnd) {
-  constexpr int kNb = (1 << BITS) - 1;
+template <int D, bool KEY>
+struct FixCfg {
+  static constexpr size_t kMat = sizeof(float) * size_t(D) * D;
+  static constexpr size_t kOffS = kMat;
+  static constexpr size_t kOffScr = kOffS + (KEY ? kMat : 0);
+  static constexpr size_t kScr = sizeof(double) * size_t(kFixBatch) * D;  // per warp
+  static constexpr size_t kOffList = kOffScr + kScr * kFixWarps;
+  static constexpr size_t kBytes = kOffList + sizeof(uint16_t) * kFixList;
+};
+
+// M^T staged as [k][lane][c] = M[32 c + lane][k]. The lanes of a warp read 16
+// bytes each from consecutive rows of M and write with stride G words.
+template <int D>
+__device__ __forceinline__ void stage_transposed(float* dst, const float* __restrict__ M) {
   constexpr int G = D / 32;
-  const int lane = threadIdx.x & 31;
-  double xk[G];
-  lane_x<D>(a.x + v * a.row_stride, xk);
-  double nn = 0.0;
-#pragma unroll
-  for (int u = 0; u < G; ++u) nn = fma(xk[u], xk[u], nn);
-  const double n64 = sqrt(warp_sum(nn));
-  // y_j, code_j and r_j for j = 32 g + lane.
-  double r[G];
-  uint32_t* idx = reinterpret_cast<uint32_t*>(a.idx + v * (D * BITS / 8));
-#pragma unroll 1
-  for (int g = 0; g < G; ++g) {
-    double part[32];
-#pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const float* row = Pis + (32 * g + m) * D + G * lane;
-      double acc = 0.0;
-#pragma unroll
-      for (int u = 0; u < G; ++u) acc = fma(static_cast<double>(row[u]), xk[u], acc);
-      part[m] = acc;
-    }
-    const double y = transpose_reduce32(part);
-    const uint32_t c = static_cast<uint32_t>(exact_code<kNb>(y, n64, bnd));
-    r[g] = y - n64 * static_cast<double>(cent[c]);
-    // Codes of this group -> BITS packed words (little-endian bit stream).
-    const int o = BITS * lane;
-#pragma unroll
-    for (int w = 0; w < BITS; ++w) {
-      uint32_t val = 0u;
-      if ((o >> 5) == w) val |= c << (o & 31);
-      if ((o >> 5) == w - 1 && (o & 31) + BITS > 32) val |= c >> (32 - (o & 31));
-      const uint32_t word = __reduce_or_sync(0xffffffffu, val);
-      if (lane == 0) idx[g * BITS + w] = word;
-    }
-  }
-  if (lane == 0) a.norm[v] = static_cast<float>(n64);
-  if (KEY) {
-    double rr = 0.0;
-#pragma unroll
-    for (int g = 0; g < G; ++g) rr = fma(r[g], r[g], rr);
-    const double rn = sqrt(warp_sum(rr));
-#pragma unroll 1
-    for (int h = 0; h < G; ++h) {
-      double part[32];
-#pragma unroll
-      for (int m = 0; m < 32; ++m) {
-        double acc = 0.0;
-#pragma unroll
-        for (int g = 0; g < G; ++g) acc = fma(static_cast<double>(Ss[(32 * h + m) * D + 32 * g + lane]), r[g], acc);
-        part[m] = acc;
-      }
-      const double p = transpose_reduce32(part);          // lane m: p_(32 h + m)
-      const uint32_t word = __ballot_sync(0xffffffffu, p >= 0.0);
-      if (lane == 0) a.sign[v * G + h] = word;
-    }
-    if (lane == 0) a.rnorm[v] = static_cast<float>(rn);
+  for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) {
+    const int i = e % D, k4 = e / D;
+    const float4 f = __ldg(reinterpret_cast<const float4*>(M + i * D) + k4);
+    const int l = i & 31, c = i >> 5;
+    dst[((4 * k4 + 0) * 32 + l) * G + c] = f.x;
+    dst[((4 * k4 + 1) * 32 + l) * G + c] = f.y;
+    dst[((4 * k4 + 2) * 32 + l) * G + c] = f.z;
+    dst[((4 * k4 + 3) * 32 + l) * G + c] = f.w;
   }
 }
 
-template <int D, bool KEY>
-constexpr size_t fix_smem_bytes() {
-  return sizeof(float) * size_t(D) * D * (KEY ? 2 : 1) + sizeof(int) * kFixList;
+// out[r][c] = sum_k M[32 c + lane][k] v_r[k] for the n rows of the batch, fp64.
+template <int D>
+__device__ __forceinline__ void batch_matvec(const float* MT, const double* scr, int n,
+                                             double (&out)[kFixBatch][D / 32]) {
+  constexpr int G = D / 32;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int r = 0; r < kFixBatch; ++r)
+#pragma unroll
+    for (int c = 0; c < G; ++c) out[r][c] = 0.0;
+#pragma unroll 4
+  for (int k = 0; k < D; ++k) {
+    double w[G];
+    if constexpr (G == 4) {
+      const float4 f = reinterpret_cast<const float4*>(MT)[k * 32 + lane];
+      w[0] = f.x; w[1] = f.y; w[2] = f.z; w[3] = f.w;
+    } else {
+      const float2 f = reinterpret_cast<const float2*>(MT)[k * 32 + lane];
+      w[0] = f.x; w[1] = f.y;
+    }
+#pragma unroll
+    for (int r = 0; r < kFixBatch; ++r) {
+      if (r < n) {
+        const double v = scr[r * D + k];
+#pragma unroll
+        for (int c = 0; c < G; ++c) out[r][c] = fma(w[c], v, out[r][c]);
+      }
+    }
+  }
+}
+
+template <int D, bool KEY, int BITS>
+__device__ __forceinline__ void fix_batch(const TcArgs& a, const int64_t (&rows)[kFixBatch], int n, const float* PiT,
+                                          const float* ST, double* scr, const float* cent, const float* bnd) {
+  constexpr int kNb = (1 << BITS) - 1;
+  constexpr int G = D / 32;
+  const int lane = threadIdx.x & 31;
+  // x of every row as fp64 into the scratch, and ||x||.
+  double n64[kFixBatch];
+#pragma unroll
+  for (int r = 0; r < kFixBatch; ++r) {
+    double nn = 0.0;
+    if (r < n) {
+      const __nv_bfloat16* xr = a.x + rows[r] * a.row_stride;
+#pragma unroll
+      for (int c = 0; c < G; ++c) {
+        const double xv = static_cast<double>(__bfloat162float(xr[32 * c + lane]));
+        scr[r * D + 32 * c + lane] = xv;
+        nn = fma(xv, xv, nn);
+      }
+    }
+    n64[r] = sqrt(warp_sum(nn));
+  }
+  __syncwarp();
+  double y[kFixBatch][G];
+  batch_matvec<D>(PiT, scr, n, y);
+  __syncwarp();                                          // x is dead: the scratch takes r
+#pragma unroll
+  for (int r = 0; r < kFixBatch; ++r) {
+    if (r >= n) continue;
+    uint32_t* idx = reinterpret_cast<uint32_t*>(a.idx + rows[r] * (D * BITS / 8));
+    double rr = 0.0;
+#pragma unroll
+    for (int c = 0; c < G; ++c) {
+      const uint32_t code = static_cast<uint32_t>(exact_code<kNb>(y[r][c], n64[r], bnd));
+      if (KEY) {
+        const double res = y[r][c] - n64[r] * static_cast<double>(cent[code]);
+        scr[r * D + 32 * c + lane] = res;
+        rr = fma(res, res, rr);
+      }
+      // Coordinates 32 c .. 32 c + 31 fill packed words c BITS .. c BITS + BITS - 1.
+      const int o = BITS * lane;
+#pragma unroll
+      for (int w = 0; w < BITS; ++w) {
+        uint32_t val = 0u;
+        if ((o >> 5) == w) val |= code << (o & 31);
+        if ((o >> 5) == w - 1 && (o & 31) + BITS > 32) val |= code >> (32 - (o & 31));
+        const uint32_t word = __reduce_or_sync(0xffffffffu, val);
+        if (lane == w) idx[c * BITS + w] = word;
+      }
+    }
+    if (lane == 0) a.norm[rows[r]] = static_cast<float>(n64[r]);
+    if (KEY) {
+      const double rn = sqrt(warp_sum(rr));
+      if (lane == 0) a.rnorm[rows[r]] = static_cast<float>(rn);
+    }
+  }
+  if (KEY) {
+    __syncwarp();
+    double pv[kFixBatch][G];
+    batch_matvec<D>(ST, scr, n, pv);
+#pragma unroll
+    for (int r = 0; r < kFixBatch; ++r) {
+      if (r >= n) continue;
+#pragma unroll
+      for (int c = 0; c < G; ++c) {
+        const uint32_t word = __ballot_sync(0xffffffffu, pv[r][c] >= 0.0);
+        if (lane == c) a.sign[rows[r] * G + c] = word;
+      }
+    }
+  }
+  __syncwarp();                                          // scratch reused by the next batch
 }
 
 template <int D, bool KEY, int BITS>
 __global__ void __launch_bounds__(kFixThreads, 1) quantize_fixup(TcArgs a) {
-  extern __shared__ __align__(16) float fix_smem[];
-  float* Pis = fix_smem;                               // [D][D]
-  float* Ss = Pis + D * D;                             // [D][D] (keys)
-  int* list = reinterpret_cast<int*>(Ss + (KEY ? D * D : 0));
+  using F = FixCfg<D, KEY>;
+  extern __shared__ __align__(16) unsigned char fix_smem[];
+  float* PiT = reinterpret_cast<float*>(fix_smem);
+  float* ST = reinterpret_cast<float*>(fix_smem + F::kOffS);
+  uint16_t* list = reinterpret_cast<uint16_t*>(fix_smem + F::kOffList);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  double* scr = reinterpret_cast<double*>(fix_smem + F::kOffScr + F::kScr * warp);
   __shared__ float cent_s[16], bnd_s[16];
   __shared__ int cnt, taken;
   if (threadIdx.x < 16) {
     cent_s[threadIdx.x] = threadIdx.x <= (1 << BITS) - 1 ? a.cent[threadIdx.x] : 0.f;
     bnd_s[threadIdx.x] = threadIdx.x < (1 << BITS) - 1 ? a.bnd[threadIdx.x] : 0.f;
   }
-  const int lane = threadIdx.x & 31;
   const float* flagp = KEY ? a.rnorm : a.norm;
   const int64_t per = (a.n + gridDim.x - 1) / gridDim.x;
   const int64_t r0 = int64_t(blockIdx.x) * per;
@@ -693,25 +730,27 @@ __global__ void __launch_bounds__(kFixThreads, 1) quantize_fixup(TcArgs a) {
       }
 #pragma unroll
       for (int u = 0; u < kPer; ++u)
-        if (fw[u] >> 31) list[atomicAdd(&cnt, 1)] = static_cast<int>(threadIdx.x + u * kFixThreads);
+        if (fw[u] >> 31) list[atomicAdd(&cnt, 1)] = static_cast<uint16_t>(threadIdx.x + u * kFixThreads);
     }
     __syncthreads();
     const int total = cnt;
     if (total == 0) continue;
     if (!staged) {
-      for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) {
-        reinterpret_cast<float4*>(Pis)[e] = __ldg(reinterpret_cast<const float4*>(a.Pi) + e);
-        if (KEY) reinterpret_cast<float4*>(Ss)[e] = __ldg(reinterpret_cast<const float4*>(a.S) + e);
-      }
+      stage_transposed<D>(PiT, a.Pi);
+      if (KEY) stage_transposed<D>(ST, a.S);
       __syncthreads();
       staged = true;
     }
     for (;;) {
       int e = 0;
-      if (lane == 0) e = atomicAdd(&taken, 1);
+      if (lane == 0) e = atomicAdd(&taken, kFixBatch);
       e = __shfl_sync(0xffffffffu, e, 0);
       if (e >= total) break;
-      fix_row<D, KEY, BITS>(a, w0 + list[e], Pis, Ss, cent_s, bnd_s);
+      const int n = total - e < kFixBatch ? total - e : kFixBatch;
+      int64_t rows[kFixBatch];
+#pragma unroll
+      for (int r = 0; r < kFixBatch; ++r) rows[r] = w0 + list[e + (r < n ? r : 0)];
+      fix_batch<D, KEY, BITS>(a, rows, n, PiT, ST, scr, cent_s, bnd_s);
     }
     __syncthreads();
   }
@@ -750,7 +789,8 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& map, cudaStream_t st) 
   quantize_tc_kernel<D, KEY, BITS><<<grid, kThreads, C::kSmemBytes, st>>>(map, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  constexpr size_t fix_smem = fix_smem_bytes<D, KEY>();
+  constexpr size_t fix_smem = FixCfg<D, KEY>::kBytes;
+  static_assert(FixCfg<D, KEY>::kBytes <= 232448, "fixup shared memory plan exceeds 227 KB");
   e = cudaFuncSetAttribute(quantize_fixup<D, KEY, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(fix_smem));
   if (e != cudaSuccess) return e;
