@@ -45,10 +45,15 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "decode-attn keys scored/s & HBM GB/s on 3+1-bit KV; quantize tokens/s"
-# DRAM bytes (read + write) per call from the ncu captures summarised under
-# profiles/ (context-8192 case, scaled x4 to the 32768-token call; traffic grows
-# with the vectors processed). None until measured for the current kernels.
-NCU_TRAFFIC = {"quantize_key": None, "quantize_value": None, "decode": None}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per call, summed
+# over the call's kernels, from one ncu capture of the full-size workload (the
+# two counters alone: one pass per launch; layer 0 of the timed step), summarised
+# in profiles/traffic_llama_full_step.md. Only reported for the full workload.
+NCU_TRAFFIC = {
+    "quantize_key": 537_350_000 + 133_300_000 + 10_240_000 + 5_120,        # main + fixup
+    "quantize_value": 537_010_000 + 90_420_000 + 9_310_000,               # main + fixup
+    "decode": 240_380 + 260_420_000 + 3_150_000 + 4_380_000,              # prologue + main + combine
+}
 
 WORKLOAD = ("Llama-3.1-8B-shaped decode: 32 layers, batch 8, 32 q / 8 kv heads, head_dim 128, context 32768, "
             "bf16 N(0,1) K/V with 2% channels x10; 3-bit+QJL keys, 3-bit values")
@@ -333,13 +338,15 @@ def run_ours(args, world, rank):
                        "call_us": 1e3 * dl_ms},
         },
         # The dominant call of the step: tq_quantize_kv of one layer's keys
-        # (quantize_tc_kernel<128, key, 3> + quantize_fixup), 2,097,152 vectors.
+        # (quantize_tc_kernel<128, key, 3> + quantize_fixup).
         "roofline": roof("tq_quantize_kv(keys): quantize_tc_kernel<128,key,3> + quantize_fixup", k_call_gbs,
-                         "bf16 in 256 B + packed out 72 B per key vector; 2,097,152 vectors per call", "quantize_key"),
+                         f"bf16 in 256 B + packed out 72 B per key vector; {n_vec:,} vectors per call",
+                         "quantize_key"),
         "roofline_value": roof("tq_quantize_kv(values): quantize_tc_kernel<128,value,3> + quantize_fixup",
-                               v_call_gbs, "bf16 in 256 B + packed out 52 B per value vector", "quantize_value"),
+                               v_call_gbs, f"bf16 in 256 B + packed out 52 B per value vector; {n_vec:,} per call",
+                               "quantize_value"),
         "roofline_decode": roof("tq_decode_attention: decode_prologue + decode_tc_kernel<3> + decode_combine",
-                                d_call_gbs, "124 B per (token, kv head); 2,097,152 per call", "decode"),
+                                d_call_gbs, f"124 B per (token, kv head); {n_vec:,} per call", "decode"),
         "clocks": clk,
         # kernels per layer: 2 (key quantize + fixup) + 2 (values) + 3 (decode)
         "gpu_launches": args.steps * L * 7,
