@@ -367,21 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         break;
       }
       tc_fence_after();
-      // The whole accumulator row in registers, one wait for the four loads.
-      // Values: the whole accumulator row in registers (one wait), after
-      // which the slot can take the next Y. Keys: two chunks per wait, and
-      // the row is read again for the codes (fewer registers live).
-      constexpr int kGrp1 = KEY ? (C::kChunks >= 2 ? 2 : 1) : C::kChunks;
-      uint32_t yb[D];
+      // Pass 1: ||y||^2, one 32-column chunk per wait (the loop is not
+      // unrolled across chunks, which keeps the epilogue in the i-cache).
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-      for (int ch0 = 0; ch0 < C::kChunks; ch0 += kGrp1) {
-#pragma unroll
-        for (int u = 0; u < kGrp1; ++u)
-          tmem_ld32(lane_addr + (ch0 + u) * 32, *reinterpret_cast<uint32_t(*)[32]>(yb + (ch0 + u) * 32));
+#pragma unroll 1
+      for (int ch = 0; ch < C::kChunks; ++ch) {
+        uint32_t yb[32];
+        tmem_ld32(lane_addr + ch * 32, yb);
         tmem_ld_wait();
 #pragma unroll
-        for (int k = ch0 * 32; k < (ch0 + kGrp1) * 32; k += 4) {
+        for (int k = 0; k < 32; k += 4) {
           const float y0 = __uint_as_float(yb[k]), y1 = __uint_as_float(yb[k + 1]);
           const float y2 = __uint_as_float(yb[k + 2]), y3 = __uint_as_float(yb[k + 3]);
           s0 = fmaf(y0, y0, s0);
@@ -389,11 +384,6 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           s2 = fmaf(y2, y2, s2);
           s3 = fmaf(y3, y3, s3);
         }
-      }
-      if (!KEY) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&accfree[wg]);
       }
       const float nrm = sqrtf((s0 + s1) + (s2 + s3));
       const float band = kCodeGuard * nrm;
@@ -410,79 +400,71 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         }
       }
       bool rowflag = false;                  // any coordinate or sign near its decision
-      uint32_t codew[C::kChunks][BITS];
       float rsq = 0.f;
-#pragma unroll
+      uint8_t* dst = a.idx + v * kRowBytes;
+      // Pass 2, per chunk: codes (stored as the chunk's BITS words), and for
+      // keys the fp16 splits of r 2^k into TMEM.
+#pragma unroll 1
       for (int ch = 0; ch < C::kChunks; ++ch) {
-        if constexpr (KEY) {
-          constexpr int kGrp = C::kChunks >= 2 ? 2 : 1;
-          if (ch % kGrp == 0) {
+        uint32_t yb[32];
+        tmem_ld32(lane_addr + ch * 32, yb);
+        tmem_ld_wait();
+        uint32_t cw[BITS];
 #pragma unroll
-            for (int u = 0; u < kGrp; ++u)
-              tmem_ld32(lane_addr + (ch + u) * 32, *reinterpret_cast<uint32_t(*)[32]>(yb + (ch + u) * 32));
-            tmem_ld_wait();
+        for (int w = 0; w < BITS; ++w) cw[w] = 0u;
+        uint32_t r1[16], r2[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          float rr[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float y = __uint_as_float(yb[k + e]);
+            const int c = code_guarded<BITS>(y, th, band, rowflag);
+            const int bp = (k + e) * BITS;
+            cw[bp >> 5] |= static_cast<uint32_t>(c) << (bp & 31);
+            if ((bp & 31) + BITS > 32) cw[(bp >> 5) + 1] |= static_cast<uint32_t>(c) >> (32 - (bp & 31));
+            rr[e] = KEY ? fmaf(-nrm, cent_s[c], y) : 0.f;
           }
-        }
-        int code[32];
-        float r[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float y = __uint_as_float(yb[ch * 32 + k]);
-          const int c = code_guarded<BITS>(y, th, band, rowflag);
-          code[k] = c;
-          if (KEY) r[k] = fmaf(-nrm, cent_s[c], y);
-        }
-#pragma unroll
-        for (int w = 0; w < BITS; ++w) codew[ch][w] = 0u;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int bp = k * BITS;
-          codew[ch][bp >> 5] |= static_cast<uint32_t>(code[k]) << (bp & 31);
-          if ((bp & 31) + BITS > 32) codew[ch][(bp >> 5) + 1] |= static_cast<uint32_t>(code[k]) >> (32 - (bp & 31));
-        }
-        if (KEY) {
-          uint32_t r1[16], r2[16];
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            rsq = fmaf(r[k], r[k], fmaf(r[k + 1], r[k + 1], rsq));
-            const float a0 = r[k] * rscale, a1 = r[k + 1] * rscale;
+          if (KEY) {
+            rsq = fmaf(rr[0], rr[0], fmaf(rr[1], rr[1], rsq));
+            const float a0 = rr[0] * rscale, a1 = rr[1] * rscale;
             const __half2 h = __floats2half2_rn(a0, a1);
             const float2 hf = __half22float2(h);
             const __half2 l = __floats2half2_rn(a0 - hf.x, a1 - hf.y);
             r1[k / 2] = *reinterpret_cast<const uint32_t*>(&h);
             r2[k / 2] = *reinterpret_cast<const uint32_t*>(&l);
           }
+        }
+        if (KEY) {
           tmem_st16(lane_addr + C::kColR1 + ch * 16, r1);
           tmem_st16(lane_addr + C::kColR2 + ch * 16, r2);
         }
+        if (valid) {
+          // The chunk's 4 BITS bytes at byte 4 BITS ch of the row.
+          uint32_t* cdst = reinterpret_cast<uint32_t*>(dst + ch * 4 * BITS);
+          if constexpr (BITS == 4) {
+            reinterpret_cast<uint4*>(cdst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          } else if constexpr (BITS == 2) {
+            reinterpret_cast<uint2*>(cdst)[0] = make_uint2(cw[0], cw[1]);
+          } else {
+#pragma unroll
+            for (int w = 0; w < BITS; ++w) cdst[w] = cw[w];
+          }
+        }
       }
-      if (KEY) {
+      if (!KEY) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accfree[wg]);
+        // Values: a row with an undecided code is flagged by the sign bit of
+        // its norm; quantize_fixup redoes it.
+        if (valid) a.norm[v] = rowflag ? -nrm : nrm;
+      } else {
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&rfull[wg]);
-      }
-      // Stores of the row's codes and norm (overlap the projection MMA).
-      if (valid) {
-        uint32_t flat[kRowBytes / 4];
-#pragma unroll
-        for (int ch = 0; ch < C::kChunks; ++ch)
-#pragma unroll
-          for (int w = 0; w < BITS; ++w) flat[ch * BITS + w] = codew[ch][w];
-        uint8_t* dst = a.idx + v * kRowBytes;
-        if constexpr (kRowBytes % 16 == 0) {
-#pragma unroll
-          for (int u = 0; u < kRowBytes / 16; ++u)
-            reinterpret_cast<uint4*>(dst)[u] = make_uint4(flat[4 * u], flat[4 * u + 1], flat[4 * u + 2], flat[4 * u + 3]);
-        } else {
-#pragma unroll
-          for (int u = 0; u < kRowBytes / 8; ++u) reinterpret_cast<uint2*>(dst)[u] = make_uint2(flat[2 * u], flat[2 * u + 1]);
-        }
-        // Values: a row with an undecided code is flagged by the sign bit of
-        // its norm (keys carry the flag on ||r||); quantize_fixup redoes it.
-        a.norm[v] = (!KEY && rowflag) ? -nrm : nrm;
-      }
-      if (KEY) {
+        if (valid) a.norm[v] = nrm;
         const float rn = sqrtf(rsq);
         const float sband = kSignGuard * rn * rscale;
         if (!__all_sync(0xffffffffu, mbar_wait(&pfull[wg], ph))) {
@@ -490,41 +472,26 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           break;
         }
         tc_fence_after();
-        uint32_t words[C::kChunks];
-        uint32_t pb[D];
-#pragma unroll
+#pragma unroll 1
         for (int ch = 0; ch < C::kChunks; ++ch) {
-          constexpr int kGrp = C::kChunks >= 2 ? 2 : 1;        // two chunks per wait
-          if (ch % kGrp == 0) {
-#pragma unroll
-            for (int u = 0; u < kGrp; ++u)
-              tmem_ld32(lane_addr + (ch + u) * 32, *reinterpret_cast<uint32_t(*)[32]>(pb + (ch + u) * 32));
-            tmem_ld_wait();
-          }
+          uint32_t pb[32];
+          tmem_ld32(lane_addr + ch * 32, pb);
+          tmem_ld_wait();
           uint32_t word = 0;
           bool near = false;
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const float p = __uint_as_float(pb[ch * 32 + k]);
+            const float p = __uint_as_float(pb[k]);
             word |= (p >= 0.f ? 1u : 0u) << k;
             near |= fabsf(p) < sband;
           }
           rowflag |= near;
-          words[ch] = word;
+          if (valid) a.sign[v * C::kChunks + ch] = word;
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&accfree[wg]);
-        if (valid) {
-          uint32_t* sdst = a.sign + v * C::kChunks;
-          if constexpr (C::kChunks == 4) {
-            reinterpret_cast<uint4*>(sdst)[0] = make_uint4(words[0], words[1], words[2], words[3]);
-          } else {
-#pragma unroll
-            for (int ch = 0; ch < C::kChunks; ++ch) sdst[ch] = words[ch];
-          }
-          a.rnorm[v] = rowflag ? __uint_as_float(__float_as_uint(rn) | 0x80000000u) : rn;
-        }
+        if (valid) a.rnorm[v] = rowflag ? __uint_as_float(__float_as_uint(rn) | 0x80000000u) : rn;
       }
     }
   }
