@@ -204,9 +204,9 @@ __device__ __forceinline__ void limbs4(float x, int (&l)[4]) {
     x = (x - static_cast<float>(l[u])) * 128.f;
   }
 }
-// int32 accumulator -> float, exact for |x| < 2^22 (every accumulator here:
-// at most 3 limb products of 128 terms, first limbs <= 127, others <= 64).
-__device__ __forceinline__ float i2f(uint32_t x) { return __uint_as_float(x + 0x4B400000u) - 12582912.f; }
+// int32 accumulator -> float (exact: every accumulator here stays below 2^22,
+// at most 3 limb products of 128 terms with limbs <= 127 in magnitude).
+__device__ __forceinline__ float i2f(uint32_t x) { return static_cast<float>(static_cast<int32_t>(x)); }
 __device__ __forceinline__ float limb_sum4(const uint32_t* d) {
   float v = i2f(d[3]);
   v = fmaf(v, 1.f / 128.f, i2f(d[2]));
@@ -455,33 +455,45 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         }
         tc_fence_after();
         const uint32_t acol = lane_addr + kColA + b * 128;
-        // Nibble selectors of the 128 codes: word g holds codes 8g..8g+7.
-        uint32_t nib[16];
+        // 32 coordinates per iteration (KB words of codes, w[0..KB-1]; the
+        // words shift down after each one): nibble selectors, then the three
+        // limbs of each coordinate by byte permutes into 8 TMEM columns per limb.
+#pragma unroll 1
+        for (int qq = 0; qq < 4; ++qq) {
+          uint32_t xq[KB + 1];
 #pragma unroll
-        for (int g = 0; g < 16; ++g) {
-          const int off = KB * g;                 // byte offset of the group
-          const int wi = off >> 2, shf = 8 * (off & 3);
-          const uint32_t x = shf == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], shf);
-          if (KB == 3) nib[g] = nibbles3(x);
-          else if (KB == 2) nib[g] = nibbles2(x);
-          else nib[g] = x;                        // 4-bit codes are nibbles already
+          for (int u = 0; u < KB; ++u) xq[u] = w[u];
+          xq[KB] = 0u;
+          uint32_t nib[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int off = KB * g;               // byte offset of the group
+            const int wi = off >> 2, shf = 8 * (off & 3);
+            const uint32_t x = shf == 0 ? xq[wi] : __funnelshift_r(xq[wi], xq[wi + 1], shf);
+            if (KB == 3) nib[g] = nibbles3(x);
+            else if (KB == 2) nib[g] = nibbles2(x);
+            else nib[g] = x;                      // 4-bit codes are nibbles already
+          }
+#pragma unroll
+          for (int limb = 0; limb < 3; ++limb) {
+            const uint32_t(&t)[4] = limb == 0 ? k1 : (limb == 1 ? k2 : k3);
+            uint32_t v8[8];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (KB <= 3) {
+                v8[2 * g] = prmt(t[0], t[1], nib[g]);
+                v8[2 * g + 1] = prmt(t[0], t[1], nib[g] >> 16);
+              } else {
+                v8[2 * g] = lut16(t, nib[g] & 0xFFFFu);
+                v8[2 * g + 1] = lut16(t, nib[g] >> 16);
+              }
+            }
+            tmem_st8(acol + limb * 32 + qq * 8, v8);
+          }
+#pragma unroll
+          for (int u = 0; u + KB < kRbk / 4 + 1; ++u) w[u] = w[u + KB];
         }
         uint32_t v[32];
-#pragma unroll
-        for (int limb = 0; limb < 3; ++limb) {
-          const uint32_t(&t)[4] = limb == 0 ? k1 : (limb == 1 ? k2 : k3);
-#pragma unroll
-          for (int g = 0; g < 16; ++g) {
-            if (KB <= 3) {
-              v[2 * g] = prmt(t[0], t[1], nib[g]);
-              v[2 * g + 1] = prmt(t[0], t[1], nib[g] >> 16);
-            } else {
-              v[2 * g] = lut16(t, nib[g] & 0xFFFFu);
-              v[2 * g + 1] = lut16(t, nib[g] >> 16);
-            }
-          }
-          tmem_st32(acol + limb * 32, v);
-        }
         // Sign chunk: column 4 m + u = sign word u AND (0x01010101 << m).
         const uint32_t sw[4] = {sg.x, sg.y, sg.z, sg.w};
 #pragma unroll
@@ -569,25 +581,33 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         }
         unsigned char* vh = sm + Sm::kOffVh + b * Sm::kVhBytes;
         // Row `row` (token) of each limb tile: 128 coordinate bytes, M-major,
-        // 8-token atoms of 1024 bytes.
+        // 8-token atoms of 1024 bytes. 32 coordinates (12 code bytes, w[0..2])
+        // per iteration; the words shift down after each one.
         const int atom = row >> 3, r8 = row & 7;
+#pragma unroll 1
+        for (int c2 = 0; c2 < 4; ++c2) {
+          const uint32_t x4[4] = {w[0], w[1], w[2], 0u};
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {        // 16 coordinates = 6 bytes of codes
-          uint32_t o1[4], o2[4];
+          for (int cc = 0; cc < 2; ++cc) {          // 16 coordinates = 6 bytes of codes
+            uint32_t o1[4], o2[4];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {             // 8 codes per half
-            const int g = 2 * c16 + h;
-            const int off = 3 * g, wi = off >> 2, shf = 8 * (off & 3);
-            const uint32_t x = shf == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], shf);
-            const uint32_t nb = nibbles3(x);
-            o1[2 * h] = prmt(v1t[0], v1t[1], nb);
-            o1[2 * h + 1] = prmt(v1t[0], v1t[1], nb >> 16);
-            o2[2 * h] = prmt(v2t[0], v2t[1], nb);
-            o2[2 * h + 1] = prmt(v2t[0], v2t[1], nb >> 16);
+            for (int h = 0; h < 2; ++h) {           // 8 codes per half
+              const int g = 2 * cc + h;
+              const int off = 3 * g, wi = off >> 2, shf = 8 * (off & 3);
+              const uint32_t x = shf == 0 ? x4[wi] : __funnelshift_r(x4[wi], x4[wi + 1], shf);
+              const uint32_t nb = nibbles3(x);
+              o1[2 * h] = prmt(v1t[0], v1t[1], nb);
+              o1[2 * h + 1] = prmt(v1t[0], v1t[1], nb >> 16);
+              o2[2 * h] = prmt(v2t[0], v2t[1], nb);
+              o2[2 * h + 1] = prmt(v2t[0], v2t[1], nb >> 16);
+            }
+            const int c16 = 2 * c2 + cc;
+            const uint32_t off = atom * 1024 + r8 * 128 + ((c16 ^ r8) << 4);
+            *reinterpret_cast<uint4*>(vh + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+            *reinterpret_cast<uint4*>(vh + kTT * 128 + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
           }
-          const uint32_t off = atom * 1024 + r8 * 128 + ((c16 ^ r8) << 4);
-          *reinterpret_cast<uint4*>(vh + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-          *reinterpret_cast<uint4*>(vh + kTT * 128 + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+#pragma unroll
+          for (int u = 0; u < 9; ++u) w[u] = w[u + 3];
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -824,13 +844,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         const float wv = vn * inv_sp;
 #pragma unroll
         for (int r = 0; r < kRowsTc; ++r) {
-          float x = fminf(p[r] * wv, 127.f);
-#pragma unroll
-          for (int l = 0; l < 3; ++l) {
-            const float t = x + kMagic;                   // rint(x) in the low mantissa bits
-            pt[poff[3 * r + l]] = static_cast<unsigned char>(__float_as_uint(t));
-            x = (x - (t - kMagic)) * 128.f;
-          }
+          // X = rint(x 2^14) < 2^21 in the low mantissa bits; its base-128
+          // digits are the limbs: x ~ d1 + d2/128 + d3/128^2.
+          const float x = fminf(p[r] * wv, 127.f);
+          const uint32_t X = __float_as_uint(fmaf(x, 16384.f, kMagic)) - 0x4B400000u;
+          pt[poff[3 * r]] = static_cast<unsigned char>(X >> 14);
+          pt[poff[3 * r + 1]] = static_cast<unsigned char>((X >> 7) & 127u);
+          pt[poff[3 * r + 2]] = static_cast<unsigned char>(X & 127u);
         }
         fence_proxy_async_smem();
         __syncwarp();
