@@ -543,14 +543,26 @@ struct FixCfg {
 template <int D>
 __device__ __forceinline__ void stage_transposed(float* dst, const float* __restrict__ M) {
   constexpr int G = D / 32;
-  for (int e = threadIdx.x; e < D * D / 4; e += blockDim.x) {
+  constexpr int kIt = D * D / 4 / kFixThreads;   // loads per thread, all in flight at once
+  static_assert(kIt * kFixThreads * 4 == D * D, "staging covers the matrix");
+  // Every CTA starts at a different part of the matrix, so the SMs do not all
+  // read the same L2 lines at once.
+  const int rot = static_cast<int>(blockIdx.x % kIt);
+  float4 f[kIt];
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    const int e = threadIdx.x + ((it + rot) % kIt) * kFixThreads;
+    f[it] = __ldg(reinterpret_cast<const float4*>(M + (e % D) * D) + e / D);
+  }
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    const int e = threadIdx.x + ((it + rot) % kIt) * kFixThreads;
     const int i = e % D, k4 = e / D;
-    const float4 f = __ldg(reinterpret_cast<const float4*>(M + i * D) + k4);
     const int l = i & 31, c = i >> 5;
-    dst[((4 * k4 + 0) * 32 + l) * G + c] = f.x;
-    dst[((4 * k4 + 1) * 32 + l) * G + c] = f.y;
-    dst[((4 * k4 + 2) * 32 + l) * G + c] = f.z;
-    dst[((4 * k4 + 3) * 32 + l) * G + c] = f.w;
+    dst[((4 * k4 + 0) * 32 + l) * G + c] = f[it].x;
+    dst[((4 * k4 + 1) * 32 + l) * G + c] = f[it].y;
+    dst[((4 * k4 + 2) * 32 + l) * G + c] = f[it].z;
+    dst[((4 * k4 + 3) * 32 + l) * G + c] = f[it].w;
   }
 }
 
@@ -564,22 +576,37 @@ __device__ __forceinline__ void batch_matvec(const float* MT, const double* scr,
   for (int r = 0; r < kFixBatch; ++r)
 #pragma unroll
     for (int c = 0; c < G; ++c) out[r][c] = 0.0;
-#pragma unroll 4
-  for (int k = 0; k < D; ++k) {
-    double w[G];
-    if constexpr (G == 4) {
-      const float4 f = reinterpret_cast<const float4*>(MT)[k * 32 + lane];
-      w[0] = f.x; w[1] = f.y; w[2] = f.z; w[3] = f.w;
-    } else {
-      const float2 f = reinterpret_cast<const float2*>(MT)[k * 32 + lane];
-      w[0] = f.x; w[1] = f.y;
+  // Blocks of four input coordinates: every load of a block is issued before
+  // its arithmetic. Rows r >= n of the scratch hold stale values; their
+  // results are discarded by the caller.
+  (void)n;
+#pragma unroll 2
+  for (int k0 = 0; k0 < D; k0 += 4) {
+    float wf[4][G];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      if constexpr (G == 4) {
+        const float4 f = reinterpret_cast<const float4*>(MT)[(k0 + kk) * 32 + lane];
+        wf[kk][0] = f.x; wf[kk][1] = f.y; wf[kk][2] = f.z; wf[kk][3] = f.w;
+      } else {
+        const float2 f = reinterpret_cast<const float2*>(MT)[(k0 + kk) * 32 + lane];
+        wf[kk][0] = f.x; wf[kk][1] = f.y;
+      }
     }
+    double v[kFixBatch][4];
 #pragma unroll
     for (int r = 0; r < kFixBatch; ++r) {
-      if (r < n) {
-        const double v = scr[r * D + k];
+      const double2 a = reinterpret_cast<const double2*>(scr + r * D + k0)[0];
+      const double2 b = reinterpret_cast<const double2*>(scr + r * D + k0)[1];
+      v[r][0] = a.x; v[r][1] = a.y; v[r][2] = b.x; v[r][3] = b.y;
+    }
 #pragma unroll
-        for (int c = 0; c < G; ++c) out[r][c] = fma(w[c], v, out[r][c]);
+    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+      for (int c = 0; c < G; ++c) {
+        const double w = wf[kk][c];
+#pragma unroll
+        for (int r = 0; r < kFixBatch; ++r) out[r][c] = fma(w, v[r][kk], out[r][c]);
       }
     }
   }
