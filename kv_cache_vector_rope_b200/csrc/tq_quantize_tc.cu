@@ -39,6 +39,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
@@ -87,7 +88,7 @@ struct Cfg {
   // full[st], empty[st], yfull[2], rfull[2], pfull[2], accfree[2], drain
   static constexpr int kNumBars = 2 * kStages + 8 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  // misc: tmem base (4) + abort (4) + r-scale exponent shift (4) + pad (4) + cent[16] + bnd[16]
+  // misc: tmem base (4) + abort (4) + r-scale exponent shift (4) + symmetric-table flag (4) + cent[16] + bnd[16]
   static constexpr int kOffCent = kOffMisc + 16;
   static constexpr int kOffBnd = kOffCent + 64;
   static constexpr int kSmemBytes = kOffBnd + 64 + 1024;   // + alignment slack
@@ -158,6 +159,21 @@ __device__ __forceinline__ int code_guarded(float y, const float (&th)[(1 << BIT
   }
 }
 
+// 3-bit code for a symmetric table (t_{6-j} = -t_j, t_3 = 0): the sign of y
+// picks the half, |y| is searched against t_4 < t_5 < t_6, and the code is
+// 4 + m (y > 0) or 3 - m. A tie |y| = t_j, where the two rules could differ,
+// lies inside the guard band and flags the row like every other near value.
+template <int NB>
+__device__ __forceinline__ int code_symmetric3(float y, const float (&th)[NB], float band, bool& near) {
+  const float ay = fabsf(y);
+  const bool b1 = ay > th[5];
+  const float tB = b1 ? th[6] : th[4];
+  const bool b0 = ay > tB;
+  near |= (ay < band) | (fabsf(ay - th[5]) < band) | (fabsf(ay - tB) < band);
+  const int m = (b1 ? 2 : 0) | (b0 ? 1 : 0);
+  return (y > 0.f ? 4 : 3) ^ m;
+}
+
 template <int D, bool KEY, int BITS>
 __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
   using C = Cfg<D, KEY>;
@@ -179,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
   int* rshift_s = reinterpret_cast<int*>(sm + C::kOffMisc + 8);
+  int* sym_s = reinterpret_cast<int*>(sm + C::kOffMisc + 12);
   float* cent_s = reinterpret_cast<float*>(sm + C::kOffCent);
   float* bnd_s = reinterpret_cast<float*>(sm + C::kOffBnd);
 
@@ -209,6 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       ++sh;
     }
     *rshift_s = sh;
+    // Exactly symmetric 3-bit boundaries (the analytic tables are).
+    bool sy = BITS == 3 && a.bnd[3] == 0.f;
+    for (int j = 0; j < kNb; ++j) sy = sy && (a.bnd[j] == -a.bnd[kNb - 1 - j]);
+    *sym_s = sy ? 1 : 0;
     mbar_fence_init();
   }
   if (tid < 16) cent_s[tid] = tid <= kNb ? a.cent[tid] : 0.f;
@@ -356,6 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     const int row = q * 32 + lane;           // row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16) + wg * C::kSlotCols;
     const int rshift = *rshift_s;
+    const bool sym = *sym_s != 0;
     float th[kNb];
     for (int it = wg; it < my_tiles; it += 2) {
       const int64_t t = blockIdx.x + int64_t(it) * gridDim.x;
@@ -404,54 +426,63 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       uint8_t* dst = a.idx + v * kRowBytes;
       // Pass 2, per chunk: codes (stored as the chunk's BITS words), and for
       // keys the fp16 splits of r 2^k into TMEM.
-#pragma unroll 1
-      for (int ch = 0; ch < C::kChunks; ++ch) {
-        uint32_t yb[32];
-        tmem_ld32(lane_addr + ch * 32, yb);
-        tmem_ld_wait();
-        uint32_t cw[BITS];
-#pragma unroll
-        for (int w = 0; w < BITS; ++w) cw[w] = 0u;
-        uint32_t r1[16], r2[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          float rr[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float y = __uint_as_float(yb[k + e]);
-            const int c = code_guarded<BITS>(y, th, band, rowflag);
-            const int bp = (k + e) * BITS;
-            cw[bp >> 5] |= static_cast<uint32_t>(c) << (bp & 31);
-            if ((bp & 31) + BITS > 32) cw[(bp >> 5) + 1] |= static_cast<uint32_t>(c) >> (32 - (bp & 31));
-            rr[e] = KEY ? fmaf(-nrm, cent_s[c], y) : 0.f;
+      // The symmetric-codebook search (3 bits) runs when the table allows it;
+      // both loops are compiled, one runs per CTA.
+      auto pass2 = [&](auto sym_tag) {
+        constexpr bool SYM = decltype(sym_tag)::value;
+  #pragma unroll 1
+        for (int ch = 0; ch < C::kChunks; ++ch) {
+          uint32_t yb[32];
+          tmem_ld32(lane_addr + ch * 32, yb);
+          tmem_ld_wait();
+          uint32_t cw[BITS];
+  #pragma unroll
+          for (int w = 0; w < BITS; ++w) cw[w] = 0u;
+          uint32_t r1[16], r2[16];
+  #pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            float rr[2];
+  #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float y = __uint_as_float(yb[k + e]);
+              int c;
+              if constexpr (SYM) c = code_symmetric3(y, th, band, rowflag);
+              else c = code_guarded<BITS>(y, th, band, rowflag);
+              const int bp = (k + e) * BITS;
+              cw[bp >> 5] |= static_cast<uint32_t>(c) << (bp & 31);
+              if ((bp & 31) + BITS > 32) cw[(bp >> 5) + 1] |= static_cast<uint32_t>(c) >> (32 - (bp & 31));
+              rr[e] = KEY ? fmaf(-nrm, cent_s[c], y) : 0.f;
+            }
+            if (KEY) {
+              rsq = fmaf(rr[0], rr[0], fmaf(rr[1], rr[1], rsq));
+              const float a0 = rr[0] * rscale, a1 = rr[1] * rscale;
+              const __half2 h = __floats2half2_rn(a0, a1);
+              const float2 hf = __half22float2(h);
+              const __half2 l = __floats2half2_rn(a0 - hf.x, a1 - hf.y);
+              r1[k / 2] = *reinterpret_cast<const uint32_t*>(&h);
+              r2[k / 2] = *reinterpret_cast<const uint32_t*>(&l);
+            }
           }
           if (KEY) {
-            rsq = fmaf(rr[0], rr[0], fmaf(rr[1], rr[1], rsq));
-            const float a0 = rr[0] * rscale, a1 = rr[1] * rscale;
-            const __half2 h = __floats2half2_rn(a0, a1);
-            const float2 hf = __half22float2(h);
-            const __half2 l = __floats2half2_rn(a0 - hf.x, a1 - hf.y);
-            r1[k / 2] = *reinterpret_cast<const uint32_t*>(&h);
-            r2[k / 2] = *reinterpret_cast<const uint32_t*>(&l);
+            tmem_st16(lane_addr + C::kColR1 + ch * 16, r1);
+            tmem_st16(lane_addr + C::kColR2 + ch * 16, r2);
+          }
+          if (valid) {
+            // The chunk's 4 BITS bytes at byte 4 BITS ch of the row.
+            uint32_t* cdst = reinterpret_cast<uint32_t*>(dst + ch * 4 * BITS);
+            if constexpr (BITS == 4) {
+              reinterpret_cast<uint4*>(cdst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            } else if constexpr (BITS == 2) {
+              reinterpret_cast<uint2*>(cdst)[0] = make_uint2(cw[0], cw[1]);
+            } else {
+  #pragma unroll
+              for (int w = 0; w < BITS; ++w) cdst[w] = cw[w];
+            }
           }
         }
-        if (KEY) {
-          tmem_st16(lane_addr + C::kColR1 + ch * 16, r1);
-          tmem_st16(lane_addr + C::kColR2 + ch * 16, r2);
-        }
-        if (valid) {
-          // The chunk's 4 BITS bytes at byte 4 BITS ch of the row.
-          uint32_t* cdst = reinterpret_cast<uint32_t*>(dst + ch * 4 * BITS);
-          if constexpr (BITS == 4) {
-            reinterpret_cast<uint4*>(cdst)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          } else if constexpr (BITS == 2) {
-            reinterpret_cast<uint2*>(cdst)[0] = make_uint2(cw[0], cw[1]);
-          } else {
-#pragma unroll
-            for (int w = 0; w < BITS; ++w) cdst[w] = cw[w];
-          }
-        }
-      }
+      };
+      if (BITS == 3 && sym) pass2(std::integral_constant<bool, BITS == 3>{});
+      else pass2(std::false_type{});
       if (!KEY) {
         tc_fence_before();
         __syncwarp();

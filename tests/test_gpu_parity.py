@@ -324,3 +324,42 @@ def test_tensor_core_and_cuda_core_quantize_paths(d, bits, monkeypatch):
         monkeypatch.delenv("TQ_QUANTIZE_PATH")
         for p in (p_tc, p_cc):
             P.compare_quantized(P.host_planes(p), ref, d, bits, is_key)
+
+
+# ---------------------------------------------------------------------------
+# The tensor-core quantizer searches a 3-bit table by |y| when the table is
+# exactly symmetric and by the general binary search otherwise: both against
+# the oracle, keys and values, several tiles and a ragged tail.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shift", [0.0, 0.013])
+def test_tensor_core_quantize_symmetric_and_shifted_tables(shift):
+    d, bits = 128, 3
+    b = ocb.lloyd_max_beta(d, bits)
+    c = np.asarray(b.centroids, dtype=np.float64)
+    c = 0.5 * (c - c[::-1])                              # exactly antisymmetric levels
+    c = c + shift / np.sqrt(d)                           # a shift breaks the symmetry
+    c32 = c.astype(np.float32)
+    t32 = (0.5 * (c[1:] + c[:-1])).astype(np.float32)
+    if shift == 0.0:
+        assert np.all(t32 == -t32[::-1]) and t32[3] == 0.0
+    else:
+        assert not np.all(t32 == -t32[::-1])
+    rg = np.random.default_rng(7)
+    n = 128 * 9 + 5
+    X = rg.standard_normal((n, d))
+    X[:, rg.choice(d, 3, replace=False)] *= 10.0
+    X[3] = 0.0
+    Xb = synth.to_bf16(X.astype(np.float32))
+    X64 = Xb.float().numpy().astype(np.float64)
+    Pi = synth.random_rotation(d, 5)
+    S = synth.gaussian_projection(d, 5)
+    lay = tq.layout(d, bits, bits)
+    for is_key in (True, False):
+        ref = oq.quantize(X64, Pi, c32.astype(np.float64), t32.astype(np.float64), bits, S=S if is_key else None)
+        planes = tq.alloc_planes(n, d, bits, is_key)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        tq.tq_quantize_kv(lay, is_key, Xb.cuda(), planes, dev(Pi), dev(c32), dev(t32),
+                          S=dev(S) if is_key else None, d_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        P.compare_quantized(P.host_planes(planes), ref, d, bits, is_key)
