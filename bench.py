@@ -130,15 +130,19 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # Distributed plumbing (one process per GPU; no data-path collective).
 # ---------------------------------------------------------------------------
-def dist_setup(args):
+def dist_setup(args=None, timeout_s: float = 600.0):
+    """One process per GPU (NCCL); without a GPU the same plumbing runs on gloo."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                             device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=timeout_s),
+                                                 device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group("gloo", timeout=datetime.timedelta(seconds=timeout_s))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -150,11 +154,18 @@ def barrier(world):
 
 
 def max_over_ranks(world, x: float) -> float:
+    """The slowest rank's time (every rank takes part)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    nccl = torch.distributed.get_backend() == "nccl"
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if nccl else "cpu")
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(rank: int) -> int:
+    """Each rank quantises and attends over its own cache (independent units)."""
+    return rank
 
 
 # ---------------------------------------------------------------------------
@@ -234,7 +245,7 @@ def run_ours(args, world, rank):
     td = torch.as_tensor(t, device=dev)
     Pi = torch.as_tensor(synth.random_rotation(D, 0), device=dev)
     S = torch.as_tensor(synth.gaussian_projection(D, 0), device=dev)
-    seed = rank  # each rank its own cache: independent units, no collective
+    seed = replica_seed(rank)  # each rank its own cache: independent units, no collective
     K = [synth.llama_layer_kv(shape, seed, l, dev, "K").reshape(n_vec, D) for l in range(L)]
     V = [synth.llama_layer_kv(shape, seed, l, dev, "V").reshape(n_vec, D) for l in range(L)]
     Q = synth.llama_queries(shape, seed, dev)[:L].reshape(L, B, HQ, 1, D).contiguous()

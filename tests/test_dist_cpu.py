@@ -1,0 +1,51 @@
+"""Multi-process plumbing of bench.py on CPU (gloo, two ranks).
+
+The hot path shards into independent (batch, kv head) units, so the ranks run
+replicas with no data-path collective; what they share is the barrier around the
+timed region and the maximum of their times. Both are checked here without a GPU.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world)})
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r, _ = bench.dist_setup(None, timeout_s=60.0)
+    try:
+        bench.barrier(w)
+        # Rank r "took" 1.5 (r + 1) ms: every rank must report the slowest.
+        slowest = bench.max_over_ranks(w, 1.5 * (r + 1))
+        seed = bench.replica_seed(r)
+        bench.barrier(w)
+        with open(os.path.join(out_dir, f"rank{r}.txt"), "w") as f:
+            f.write(f"{w} {r} {slowest} {seed} {torch.distributed.get_backend()}\n")
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the gloo path; GPU runs use NCCL")
+def test_two_rank_barrier_max_and_replica_seeds(tmp_path):
+    world = 2
+    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    rows = [open(tmp_path / f"rank{r}.txt").read().split() for r in range(world)]
+    for r, (w, rank, slowest, seed, backend) in enumerate(rows):
+        assert int(w) == world and int(rank) == r
+        assert float(slowest) == 1.5 * world          # max over ranks, seen by every rank
+        assert backend == "gloo"
+    assert len({row[3] for row in rows}) == world       # independent caches per rank

@@ -363,3 +363,59 @@ def test_tensor_core_quantize_symmetric_and_shifted_tables(shift):
         torch.cuda.synchronize()
         assert int(st.item()) == 0
         P.compare_quantized(P.host_planes(planes), ref, d, bits, is_key)
+
+
+# ---------------------------------------------------------------------------
+# Guard canaries: every output buffer sits between 4 KiB fences of a known byte;
+# after quantize (ragged tail), decode and dequantize the fences must be intact.
+# ---------------------------------------------------------------------------
+_FENCE = 4096
+
+
+def _fenced(shape, dtype):
+    n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+    buf = torch.full((2 * _FENCE + n,), 0xA5, dtype=torch.uint8, device="cuda")
+    return buf, buf[_FENCE:_FENCE + n].view(dtype).view(*shape)
+
+
+def _fences_intact(buf):
+    return bool((buf[:_FENCE] == 0xA5).all()) and bool((buf[buf.numel() - _FENCE:] == 0xA5).all())
+
+
+def test_output_fences_intact_after_quantize_decode_dequantize():
+    d, bits, B, HKV, HQ, N = 128, 3, 2, 2, 8, 1000     # tensor-core paths, ragged tiles
+    n = B * HKV * N
+    c32, t32 = book(d, bits)
+    Pi = synth.random_rotation(d, 11)
+    S = synth.gaussian_projection(d, 11)
+    rg = np.random.default_rng(11)
+    X = synth.to_bf16(rg.standard_normal((2, n, d)).astype(np.float32)).cuda()
+    lay = tq.layout(d, bits, bits)
+    bufs = []
+
+    def fenced_planes(is_key):
+        fb = [_fenced((n, tq.tq_idx_row_bytes(d, bits)), torch.uint8), _fenced((n,), torch.float32)]
+        if is_key:
+            fb += [_fenced((n, tq.tq_sign_words(d)), torch.int32), _fenced((n,), torch.float32)]
+        bufs.extend(b for b, _ in fb)
+        v = [t for _, t in fb]
+        return tq.Planes(idx=v[0], norm=v[1], sign=v[2] if is_key else None, rnorm=v[3] if is_key else None)
+
+    kp, vp = fenced_planes(True), fenced_planes(False)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.tq_quantize_kv(lay, True, X[0], kp, dev(Pi), dev(c32), dev(t32), S=dev(S), d_status=st)
+    tq.tq_quantize_kv(lay, False, X[1], vp, dev(Pi), dev(c32), dev(t32), d_status=st)
+    q = torch.randn(B, HQ, 1, d, device="cuda")
+    ob, out = _fenced((B, HQ, 1, d), torch.float32)
+    ws_bytes = (tq.tq_decode_workspace_bytes(lay, B, HQ, HKV, 1, N) + 255) // 256 * 256
+    wb, ws = _fenced((ws_bytes,), torch.uint8)
+    sb, scores = _fenced((B, HQ, 1, N), torch.float32)
+    tq.tq_decode_attention(lay, q, kp, vp, HKV, N, dev(Pi), dev(Pi), dev(S), dev(c32), dev(c32), out, ws,
+                           scores_out=scores, d_status=st)
+    db, deq = _fenced((n, d), torch.float32)
+    tq.tq_dequantize(lay, True, kp, n, dev(Pi), dev(c32), deq, S=dev(S))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    bufs += [ob, wb, sb, db]
+    assert all(_fences_intact(b) for b in bufs)
+    assert torch.isfinite(out).all() and torch.isfinite(deq).all()
