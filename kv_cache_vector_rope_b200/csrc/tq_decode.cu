@@ -549,11 +549,10 @@ __global__ void __launch_bounds__(kBlkThreads) decode_combine(DecodeArgs a, RowB
 }
 
 // ---------------------------------------------------------------------------
-// Few query rows (the GQA decode shape): one warp per row, the matrices read
-// straight from L2 (no staging), so the prologue and the combine spread over
-// many SMs. Lane l owns the G = d/32 coordinates it loads and writes.
+// Few query rows (the GQA decode shape): one CTA of d threads per row, the
+// matrices read straight from L2 (no staging), so the prologue and the
+// combine spread over many SMs with every load coalesced.
 // ---------------------------------------------------------------------------
-constexpr int kRowWarps = 4;                 // rows (warps) per CTA
 constexpr int kRowWarpMaxRows = 512;         // above this, the row-block kernels
 
 // The row's Pi (shared, or the row's KV head's).
@@ -563,151 +562,131 @@ __device__ __forceinline__ int row_kv(const DecodeArgs& a, int64_t row) {
   return static_cast<int>((row / rows_per_group) % a.sh.hkv);
 }
 
-// out[c] = sum_j M[(lane + 32 c) d + j] v[j] for c < G, v in shared memory.
-template <int G>
-__device__ __forceinline__ void warp_matvec_rows(const float* __restrict__ M, const float* v, float (&out)[G]) {
-  constexpr int d = 32 * G;
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int c = 0; c < G; ++c) out[c] = 0.f;
-#pragma unroll 8
-  for (int j = 0; j < d; j += 4) {
-    const float4 x = *reinterpret_cast<const float4*>(v + j);
-#pragma unroll
-    for (int c = 0; c < G; ++c) {
-      const float4 m = __ldg(reinterpret_cast<const float4*>(M + (lane + 32 * c) * d + j));
-      out[c] = fmaf(m.x, x.x, fmaf(m.y, x.y, fmaf(m.z, x.z, fmaf(m.w, x.w, out[c]))));
-    }
-  }
-}
-
-template <int G>
-__global__ void __launch_bounds__(32 * kRowWarps) decode_prologue_rows(DecodeArgs a) {
-  constexpr int d = 32 * G;
-  __shared__ __align__(16) float vs[kRowWarps][d];
-  const DecodeShape& s = a.sh;
+// y[i] = sum_j M[i][j] v[j] for the D/32 rows i = 32 w + o handled by warp w:
+// lane l reads M[i][G l .. G l + G) (one coalesced row read per i) and the
+// warp sums the products. v in shared memory; y written to ys (shared) and out.
+template <int D>
+__device__ __forceinline__ void row_matvec_warps(const float* __restrict__ M, const float* v, float* ys,
+                                                 float* __restrict__ out) {
+  constexpr int G = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = int64_t(blockIdx.x) * kRowWarps + warp;
-  if (row >= s.n_rows) return;
-  const int kv = row_kv(a, row);
-  // RoPE pairs (i, i + d/2) are lane-local: coordinates lane + 32 c and
-  // lane + 32 (c + G/2).
   float x[G];
 #pragma unroll
-  for (int c = 0; c < G; ++c) x[c] = load_elem(a.q, a.q_dtype, row * d + lane + 32 * c);
-  if (a.q_pos != nullptr && a.rope_base > 0.0) {
-    int b, h, n;
-    row_coords(s, row, b, h, n);
-    const int pos = a.q_pos[int64_t(b) * s.nq + n];
-    if (pos < 0 && a.d_status && lane == 0) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
-#pragma unroll
-    for (int c = 0; c < G / 2; ++c) {
-      double sn, cs;
-      sincos(rope_angle(pos, lane + 32 * c, d, a.rope_base), &sn, &cs);
-      const double x0 = x[c], x1 = x[c + G / 2];
-      x[c] = static_cast<float>(x0 * cs - x1 * sn);
-      x[c + G / 2] = static_cast<float>(x0 * sn + x1 * cs);
+  for (int c = 0; c < G; ++c) x[c] = v[G * lane + c];
+  constexpr int kRowsPerWarp = D / (D / 32);    // 32 rows per warp (D/32 warps)
+#pragma unroll 8
+  for (int o = 0; o < kRowsPerWarp; ++o) {
+    const int i = warp * kRowsPerWarp + o;
+    float p;
+    if constexpr (G == 4) {
+      const float4 m = __ldg(reinterpret_cast<const float4*>(M + i * D) + lane);
+      p = fmaf(m.x, x[0], fmaf(m.y, x[1], fmaf(m.z, x[2], m.w * x[3])));
+    } else {
+      const float2 m = __ldg(reinterpret_cast<const float2*>(M + i * D) + lane);
+      p = fmaf(m.x, x[0], m.y * x[1]);
+    }
+    p = warp_sum(p);
+    if (lane == 0) {
+      if (ys) ys[i] = p;
+      out[i] = p;
     }
   }
-#pragma unroll
-  for (int c = 0; c < G; ++c) vs[warp][lane + 32 * c] = x[c];
-  __syncwarp();
-  float y[G];
-  warp_matvec_rows<G>(a.PiK + int64_t(kv) * a.pi_stride, vs[warp], y);
-  __syncwarp();
-#pragma unroll
-  for (int c = 0; c < G; ++c) {
-    vs[warp][lane + 32 * c] = y[c];
-    a.qs[row * 2 * d + lane + 32 * c] = y[c];
-  }
-  __syncwarp();
-  warp_matvec_rows<G>(a.S, vs[warp], y);
-#pragma unroll
-  for (int c = 0; c < G; ++c) a.qs[row * 2 * d + d + lane + 32 * c] = y[c];
 }
 
-template <int G>
-__global__ void __launch_bounds__(32 * kRowWarps) decode_combine_rows(DecodeArgs a) {
-  constexpr int d = 32 * G;
-  __shared__ __align__(16) float vs[kRowWarps][d];
+template <int D>
+__global__ void __launch_bounds__(D) decode_prologue_rows(DecodeArgs a) {
+  __shared__ __align__(16) float xs[D], ys[D];
+  const DecodeShape& s = a.sh;
+  const int64_t row = blockIdx.x;
+  const int i = threadIdx.x;
+  const int kv = row_kv(a, row);
+  // RoPE pairs (i, i + D/2).
+  if (i < D / 2) {
+    float x0 = load_elem(a.q, a.q_dtype, row * D + i);
+    float x1 = load_elem(a.q, a.q_dtype, row * D + i + D / 2);
+    if (a.q_pos != nullptr && a.rope_base > 0.0) {
+      int b, h, n;
+      row_coords(s, row, b, h, n);
+      const int pos = a.q_pos[int64_t(b) * s.nq + n];
+      if (pos < 0 && a.d_status && i == 0) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
+      double sn, cs;
+      sincos(rope_angle(pos, i, D, a.rope_base), &sn, &cs);
+      const double r0 = double(x0) * cs - double(x1) * sn, r1 = double(x0) * sn + double(x1) * cs;
+      x0 = static_cast<float>(r0);
+      x1 = static_cast<float>(r1);
+    }
+    xs[i] = x0;
+    xs[i + D / 2] = x1;
+  }
+  __syncthreads();
+  row_matvec_warps<D>(a.PiK + int64_t(kv) * a.pi_stride, xs, ys, a.qs + row * 2 * D);
+  __syncthreads();
+  row_matvec_warps<D>(a.S, ys, nullptr, a.qs + row * 2 * D + D);
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_rows(DecodeArgs a) {
+  __shared__ __align__(16) float os[D];
+  __shared__ float wk[64];
+  __shared__ float inv_l_s;
   const DecodeShape& s = a.sh;
   const int ns = s.n_parts;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = int64_t(blockIdx.x) * kRowWarps + warp;
-  if (row >= s.n_rows) return;
+  const int64_t row = blockIdx.x;
+  const int i = threadIdx.x, warp = i >> 5, lane = i & 31;
   const int kv = row_kv(a, row);
-  const float* part = a.part + row * ns * (d + 2);
-  // Row maximum and softmax denominator over the partial records.
-  float M = -INFINITY;
-  for (int k = lane; k < ns; k += 32) M = fmaxf(M, part[k * (d + 2) + d]);
-  M = warp_max(M);
-  float L = 0.f;
-  for (int k = lane; k < ns; k += 32) {
-    const float mk = part[k * (d + 2) + d];
-    if (mk > -INFINITY) L += __expf(mk - M) * part[k * (d + 2) + d + 1];
+  const float* part = a.part + row * ns * (D + 2);
+  // Row maximum and softmax denominator (warp 0); the record weights go to
+  // shared memory when they fit (else every thread forms them itself).
+  if (warp == 0) {
+    float M = -INFINITY;
+    for (int k = lane; k < ns; k += 32) M = fmaxf(M, part[k * (D + 2) + D]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int k = lane; k < ns; k += 32) {
+      const float mk = part[k * (D + 2) + D];
+      const float w = mk > -INFINITY ? __expf(mk - M) : 0.f;
+      if (k < 64) wk[k] = w;
+      L += w * part[k * (D + 2) + D + 1];
+    }
+    L = warp_sum(L);
+    if (lane == 0) inv_l_s = L > 0.f ? 1.f / L : 0.f;
+    if (lane == 0 && ns > 64) wk[0] = M;          // the reference for the slow path
   }
-  L = warp_sum(L);
-  // Merged rotated output: lane owns coordinates G lane .. G lane + G - 1
-  // (8-byte loads: a record starts on an 8-byte boundary).
-  float o[G];
-#pragma unroll
-  for (int c = 0; c < G; ++c) o[c] = 0.f;
+  __syncthreads();
+  float o = 0.f;
+  if (ns <= 64) {
 #pragma unroll 8
-  for (int k = 0; k < ns; ++k) {
-    const float mk = part[k * (d + 2) + d];
-    const float w = mk > -INFINITY ? __expf(mk - M) : 0.f;
-    const float2* rec = reinterpret_cast<const float2*>(part + k * (d + 2) + G * lane);
-#pragma unroll
-    for (int c2 = 0; c2 < G / 2; ++c2) {
-      const float2 r = rec[c2];
-      o[2 * c2] = fmaf(w, r.x, o[2 * c2]);
-      o[2 * c2 + 1] = fmaf(w, r.y, o[2 * c2 + 1]);
+    for (int k = 0; k < ns; ++k) o = fmaf(wk[k], part[k * (D + 2) + i], o);
+  } else {
+    const float M = wk[0];
+    for (int k = 0; k < ns; ++k) {
+      const float mk = part[k * (D + 2) + D];
+      if (mk > -INFINITY) o = fmaf(__expf(mk - M), part[k * (D + 2) + i], o);
     }
   }
-  const float inv_l = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-  for (int c = 0; c < G; ++c) vs[warp][G * lane + c] = o[c] * inv_l;
-  __syncwarp();
-  // out[j] = sum_i Pi_V[i][j] o[i], lane owns j = G lane .. G lane + G - 1.
+  os[i] = o * inv_l_s;
+  __syncthreads();
+  // out[j] = sum_i Pi_V[i][j] o[i], thread j (coalesced reads of row i).
   const float* PiV = a.PiV + int64_t(kv) * a.pi_stride;
-  float acc[G];
-#pragma unroll
-  for (int c = 0; c < G; ++c) acc[c] = 0.f;
+  float acc = 0.f;
 #pragma unroll 16
-  for (int i = 0; i < d; ++i) {
-    const float oi = vs[warp][i];
-    const float* prow = PiV + i * d + G * lane;
-    if constexpr (G == 4) {
-      const float4 m = __ldg(reinterpret_cast<const float4*>(prow));
-      acc[0] = fmaf(m.x, oi, acc[0]);
-      acc[1] = fmaf(m.y, oi, acc[1]);
-      acc[2] = fmaf(m.z, oi, acc[2]);
-      acc[3] = fmaf(m.w, oi, acc[3]);
-    } else {
-      const float2 m = __ldg(reinterpret_cast<const float2*>(prow));
-      acc[0] = fmaf(m.x, oi, acc[0]);
-      acc[1] = fmaf(m.y, oi, acc[1]);
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < G; ++c) {
-    const int64_t at = row * d + G * lane + c;
-    if (a.out_dtype == 0)
-      reinterpret_cast<float*>(a.out)[at] = acc[c];
-    else
-      reinterpret_cast<__nv_bfloat16*>(a.out)[at] = __float2bfloat16(acc[c]);
-  }
+  for (int r = 0; r < D; ++r) acc = fmaf(__ldg(PiV + r * D + i), os[r], acc);
+  const int64_t at = row * D + i;
+  if (a.out_dtype == 0)
+    reinterpret_cast<float*>(a.out)[at] = acc;
+  else
+    reinterpret_cast<__nv_bfloat16*>(a.out)[at] = __float2bfloat16(acc);
 }
 
 template <bool COMBINE>
 cudaError_t launch_rows(const DecodeArgs& a, cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>((a.sh.n_rows + kRowWarps - 1) / kRowWarps);
+  const unsigned grid = static_cast<unsigned>(a.sh.n_rows);
   if (a.sh.d == 128) {
-    if (COMBINE) decode_combine_rows<4><<<grid, 32 * kRowWarps, 0, st>>>(a);
-    else decode_prologue_rows<4><<<grid, 32 * kRowWarps, 0, st>>>(a);
+    if (COMBINE) decode_combine_rows<128><<<grid, 128, 0, st>>>(a);
+    else decode_prologue_rows<128><<<grid, 128, 0, st>>>(a);
   } else {
-    if (COMBINE) decode_combine_rows<2><<<grid, 32 * kRowWarps, 0, st>>>(a);
-    else decode_prologue_rows<2><<<grid, 32 * kRowWarps, 0, st>>>(a);
+    if (COMBINE) decode_combine_rows<64><<<grid, 64, 0, st>>>(a);
+    else decode_prologue_rows<64><<<grid, 64, 0, st>>>(a);
   }
   return cudaGetLastError();
 }
