@@ -52,7 +52,7 @@ METRIC = "decode-attn keys scored/s & HBM GB/s on 3+1-bit KV; quantize tokens/s"
 NCU_TRAFFIC = {
     "quantize_key": 537_220_000 + 130_370_000 + 10_240_000 + 5_380,        # main + fixup
     "quantize_value": 537_050_000 + 90_680_000 + 9_310_000 + 256,         # main + fixup
-    "decode": 240_130 + 260_450_000 + 2_820_000 + 4_380_000,              # prologue + main + combine
+    "decode": 217_600 + 260_410_000 + 4_120_000 + 4_350_000,              # prologue + main + combine
 }
 
 WORKLOAD = ("Llama-3.1-8B-shaped decode: 32 layers, batch 8, 32 q / 8 kv heads, head_dim 128, context 32768, "
