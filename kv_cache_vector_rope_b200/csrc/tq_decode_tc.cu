@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
     }
   } else if (warp == 1 || warp == 14) {
     // ------------------------------------------ MMA issuers (one thread each)
-    // warp 1 issues the score MMAs, warp 18 the PV MMAs, so the issue
+    // warp 1 issues the score MMAs, warp 14 the PV MMAs, so the issue
     // latencies of the two chains overlap.
     if (lane == 0) {
       const uint32_t id_mse = idesc_i8(true, false), id_sgn = idesc_i8(false, false), id_v = idesc_i8(true, true);
