@@ -17,10 +17,13 @@
 //                 P = (R1 + R2) (S1 + S2)^T      fp16 splits, A from TMEM
 //                                                (R2 S1 + R1 S2 + R1 S1)
 //   warps 2-5   epilogue warpgroup 0, warps 6-9 epilogue warpgroup 1; thread =
-//               vector (TMEM lane). Per tile: ||y|| from the accumulator, codes
-//               by binary search against ||y|| t_j, residual r, fp16 splits of
-//               r 2^k (k from ||y||, so r 2^k stays below 2^14) into TMEM for P,
-//               sign bits from P, packing and stores.
+//               vector (TMEM lane). Per tile, in 32-column chunks (a loop that is
+//               not unrolled across chunks, so the epilogue stays in the
+//               instruction cache): ||y|| from the accumulator; codes by binary
+//               search against ||y|| t_j (by |y| against t_4..t_6 when the
+//               3-bit table is exactly symmetric); residual r and the fp16
+//               splits of r 2^k (k from ||y||, so r 2^k stays below 2^14) into
+//               TMEM for P; sign bits from P; packing and stores per chunk.
 // TMEM slot (keys): Y/P accumulator (d columns) | R1 (d/2) | R2 (d/2).
 //
 // Exactness. The norm is ||y|| = ||Pi x|| in fp32 (Pi orthogonal; error
@@ -28,8 +31,8 @@
 // 3e-7 ||y|| from every boundary it was compared with, a sign only when |p|
 // exceeds 1.5e-5 ||r||. A row with any other coordinate or sign is flagged
 // (sign bit of its stored ||r|| for keys, of ||x|| for values) and a second
-// launch, quantize_fixup, recomputes every flagged row exactly in fp64 (one
-// warp per row: ||x||, y = Pi x, codes, r, p = S r) and overwrites it.
+// launch, quantize_fixup, recomputes every flagged row exactly in fp64 (four
+// rows per warp: ||x||, y = Pi x, codes, r, p = S r) and overwrites it.
 //
 // Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT in *d_status and
 // the CTA drains its own copies and MMAs, frees TMEM and returns.
