@@ -356,7 +356,7 @@ def run_ours(args, world, rank):
         "roofline_value": roof("tq_quantize_kv(values): quantize_tc_kernel<128,value,3> + quantize_fixup",
                                v_call_gbs, f"bf16 in 256 B + packed out 52 B per value vector; {n_vec:,} per call",
                                "quantize_value"),
-        "roofline_decode": roof("tq_decode_attention: decode_prologue + decode_tc_kernel<3> + decode_combine",
+        "roofline_decode": roof("tq_decode_attention: decode_prologue_rows + decode_tc_kernel<3> + decode_combine_rows",
                                 d_call_gbs, f"124 B per (token, kv head); {n_vec:,} per call", "decode"),
         "clocks": clk,
         # kernels per layer: 2 (key quantize + fixup) + 2 (values) + 3 (decode)
