@@ -72,9 +72,7 @@ DecodeShape make_shape(const tq_layout* L, int batch, int hq, int hkv, int nq, i
 
 size_t shape_workspace_bytes(const DecodeShape& s) {
   const size_t qs = size_t(s.n_rows) * 2 * s.d * sizeof(float);
-  // Room for two partial records per split (the tensor-core kernel splits each
-  // work item into its even and odd tiles).
-  const size_t part = size_t(s.n_rows) * 2 * s.n_splits * (s.d + 2) * sizeof(float);
+  const size_t part = size_t(s.n_rows) * s.n_splits * (s.d + 2) * sizeof(float);
   return ((qs + 255) / 256) * 256 + part;
 }
 
@@ -780,7 +778,8 @@ extern "C" size_t tq_decode_workspace_bytes(const tq_layout* layout, int32_t bat
                                             int32_t nq, int64_t n_ctx) {
   if (tq::check_layout(layout) != TQ_OK || batch < 1 || hkv < 1 || hq < hkv || hq % hkv || nq < 1 || n_ctx < 1)
     return 0;
-  return tq::shape_workspace_bytes(tq::make_shape(layout, batch, hq, hkv, nq, n_ctx, n_ctx));
+  const tq::DecodeShape sh = tq::make_shape(layout, batch, hq, hkv, nq, n_ctx, n_ctx);
+  return std::max(tq::shape_workspace_bytes(sh), tq::tc_decode_workspace_bytes(sh));
 }
 
 extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q, tq_dtype q_dtype, int32_t batch,
@@ -808,7 +807,7 @@ extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q,
   if (!aligned(k->idx, 16) || !aligned(k->sign, 16) || !aligned(v->idx, 16))
     return fail(TQ_ERR_INVALID_ARG, "plane pointers must be 16-byte aligned");
   const DecodeShape sh = make_shape(layout, batch, hq, hkv, nq, n_ctx, ctx_stride);
-  const size_t need = shape_workspace_bytes(sh);
+  const size_t need = std::max(shape_workspace_bytes(sh), tc_decode_workspace_bytes(sh));
   if (!workspace || workspace_bytes < need)
     return fail(TQ_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
   if (!aligned(workspace, 256)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
@@ -841,26 +840,24 @@ extern "C" tq_status tq_decode_attention(const tq_layout* layout, const void* q,
                                     ((size_t(sh.n_rows) * 2 * d * sizeof(float) + 255) / 256) * 256);
   a.d_status = d_status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_blk<false>(a, s);
-  if (e == cudaSuccess) {
-    // Tensor-core kernel where it applies (TQ_DECODE_PATH=v1|v2 selects a
-    // CUDA-core kernel instead; all compute the same attention).
-    const char* path = std::getenv("TQ_DECODE_PATH");
-    const bool cuda_core = path && (std::strcmp(path, "v1") == 0 || std::strcmp(path, "v2") == 0);
-    if (!cuda_core && tc_decode_supported(a)) {
-      a.sh.n_parts = 2 * a.sh.n_splits;
-      e = tc_decode_launch(a, s);
-    } else {
-    switch (d) {
-      case 64: e = launch_main_rows<64>(a, s); break;
-      case 128: e = launch_main_rows<128>(a, s); break;
-      case 200: e = launch_main_rows<200>(a, s); break;
-      default: return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: d=%d not built (64, 128, 200)", d);
+  cudaError_t e;
+  // The fused tensor-core kernel where it applies (TQ_DECODE_PATH=v1|v2
+  // selects a CUDA-core kernel instead; all compute the same attention).
+  const char* path = std::getenv("TQ_DECODE_PATH");
+  const bool cuda_core = path && (std::strcmp(path, "v1") == 0 || std::strcmp(path, "v2") == 0);
+  if (!cuda_core && tc_decode_supported(a)) {
+    e = tc_decode_launch(a, workspace, s);
+  } else {
+    e = launch_blk<false>(a, s);
+    if (e == cudaSuccess) {
+      switch (d) {
+        case 64: e = launch_main_rows<64>(a, s); break;
+        case 128: e = launch_main_rows<128>(a, s); break;
+        case 200: e = launch_main_rows<200>(a, s); break;
+        default: return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: d=%d not built (64, 128, 200)", d);
+      }
     }
-    }
-  }
-  if (e == cudaSuccess) {
-    e = launch_blk<true>(a, s);
+    if (e == cudaSuccess) e = launch_blk<true>(a, s);
   }
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_decode_attention launch: %s", cudaGetErrorString(e));
   return TQ_OK;

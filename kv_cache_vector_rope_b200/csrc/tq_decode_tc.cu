@@ -1,49 +1,54 @@
-// Tensor-core decode attention (sm_100a, tcgen05 kind::i8) for d = 128 with
-// four query rows per KV stream (the GQA decode shape) and 3-bit values.
+// Fused tensor-core decode attention (sm_100a, tcgen05 kind::i8) for d = 128,
+// four query rows per KV stream (a GQA group of four heads, one query each),
+// 3-bit values and 2-4-bit keys: the whole call in one launch.
 //
 // Sources: gist.science "TurboESM ..." section 2E (one fused kernel unpacks
 // the codes, applies the QJL correction and the inverse rotation and runs an
 // online softmax, with no dequantised tensor in memory) and 7minutos.es
 // "KV cache ... TurboQuant" Etapa 2 (the QJL estimator).
 //
-// Both contractions of decode run on the tensor cores over operands rebuilt
-// from the packed cache in on-chip memory, with exact integer arithmetic:
-//   scores  A (TMEM, one lane per token), 128 columns per tile:
-//             a1 | a2 | a3   the key codebook value of every coordinate as
-//                            three int8 limbs, c = sc (a1 + a2/128 + a3/128^2)
-//             sgn            the sign bits, masked in place: byte 16 j + b is
-//                            byte b of the sign row AND (1 << j), i.e. bit
-//                            8 b + j of the sketch times 2^j (unsigned)
-//           B (smem, K-major): per query row four int8 limbs of q_rot and of
-//           s' = s 2^-(i mod 8) (sign-chunk rows permuted to match). Limb
-//           products of equal weight 128^-w go to the same int32 column: the
-//           a1, a2, a3 chunks use B tiles whose limb columns are shifted by
-//           0, 1, 2, so D column 4 r + w holds sum_{l+m=w} a_l q_m.
-//   values  O[i][n] = sum_t c_V[code_ti] w_t,n: A (smem, M-major) the value
-//           codebook as two int8 limbs per coordinate, one 128-byte row per
-//           token; B the tile's weights w = p ||v|| / s_item as three int8
-//           limbs per query row, s_item = max ||v|| over the work item / 127
-//           (p <= 1 because the running maximum only grows).
-// Online softmax: the running maximum per row only moves when a score of the
-// tile exceeds it (a vote over the softmax warps; the tile maximum is reduced
-// only then), so an ordinary tile costs one barrier; l is kept per thread and
-// summed once per work item. The value warps fold each PV product into their
-// accumulators (thread = coordinate) with the tile's correction, which the
-// softmax warps leave in a four-slot ring.
-// Roles (480 threads, one persistent CTA per SM):
-//   warp 0     bulk copies of the packed index / sign planes into a 3-stage ring
-//   warp 1     TMEM owner and single-thread issuer of the score MMAs
-//   warp 14    single-thread issuer of the PV MMAs
-//   warps 2-5  key operand generation into TMEM        (thread = token)
-//   warps 6-9  value operand generation into smem      (thread = token)
-//             and the value epilogue                   (thread = coordinate)
-//   warps 10-13 scores, softmax and weight limbs       (thread = token); the
-//             even and odd tiles of a work item keep separate running maxima
-//             and sums, so a work item leaves two partial records
+//   Work        all (stream, 128-token tile) pairs in stream order are cut into
+//               equal contiguous ranges, one per persistent CTA (longer than
+//               512 tiles: cut again). A range splits into segments at stream
+//               ends; each segment leaves one partial record (m, l, acc) per
+//               query row.
+//   Prologue    per segment: q_rot = Pi_K RoPE(q), s = S q_rot and their int8
+//               limbs as the B operands of the score MMAs.
+//   Scores      A (TMEM, one lane per token): the key codebook value of every
+//               coordinate as three int8 limbs, c = sc (a1 + a2/128 + a3/128^2),
+//               and the sign chunk, masked in place (byte 16 j + b = byte b of
+//               the sign row AND 1 << j); B (smem): limbs of q_rot and of
+//               s' = s 2^-(i mod 8). Limb products of equal weight share an
+//               int32 column: 16 MMAs (M = 128, N = 16, K = 32) per tile.
+//   Softmax     thread = token. The running maximum m of each query row is set
+//               by the segment's first tile and only moves when a weight
+//               x = 2^(score - m) ||v|| / V0 (V0: largest ||v|| of that first
+//               tile) would exceed 64; then it moves by whole octaves. The
+//               weights are 32-bit fixed point, X = rint(x 2^24): their four
+//               bytes are the unsigned B limbs of the value MMAs, one 16-byte
+//               shared store per token (B MN-major, 16 bytes per token).
+//   Values      A (smem, MN-major): the value codebook as two int8 limbs per
+//               coordinate, one 128-byte row per token. The PV products add up
+//               in TMEM over all tiles of a segment; only when m moves (rare)
+//               is the accumulator folded into registers (thread = coordinate)
+//               and restarted in the other TMEM region.
+//   Combine     the last segment of a stream to finish (a per-stream arrival
+//               counter) merges the stream's records and applies Pi_V^T.
+// Roles (512 threads, one CTA per SM):
+//   warp 0       bulk copies of the index and sign planes into a 4-stage ring
+//   warp 1       TMEM owner and score MMA issuer   (warp-uniform loop, elected lane)
+//   warp 2       PV MMA issuer
+//   warps 4-7    key operands into TMEM            (thread = token)
+//   warps 8-11   value operands into smem, folds, combine (thread = token / coordinate)
+//   warps 12-15  scores, softmax, weights          (thread = token)
+// Warps 8-15 also compute the segment prologue together.
 // Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT and the CTA
 // drains its copies and MMAs before it frees TMEM and returns.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "tq_decode_tc.h"
 #include "tq_device.cuh"
@@ -54,74 +59,92 @@ namespace tq {
 namespace {
 
 using namespace sm100;
+using dev::load_elem;
 using dev::warp_max;
 using dev::warp_sum;
 
 constexpr int kD = 128;
 constexpr int kTT = 128;               // tokens per tile
-constexpr int kStages = 3;
-constexpr int kThreadsTc = 480;        // 15 warps
-constexpr int kRowsTc = 4;
+constexpr int kStages = 4;
+constexpr int kThreads = 640;          // 20 warps
+constexpr int kRows = 4;               // query rows per stream
+constexpr int kMaxSegTiles = 512;      // PV accumulators: < 2^31 over this many tiles
+constexpr int kMaxGrid = 256;
+constexpr int kRecFloats = 132;        // partial record: acc[128], m, l, pad
+constexpr int kWLoader = 0, kWScore = 1, kWPv = 2, kWKey0 = 4, kWVal0 = 8, kWSoft0 = 12;   // softmax groups: 12-15, 16-19
+constexpr int kSegFloats = 48;         // per-segment constants
 
 // TMEM columns (32-bit): A_score x2 at 0, 128 (a1 | a2 | a3 | sgn, 32 each);
-// D_score x2 at 256, 288 (mse 16 | sgn 16); D_o x2 at 320, 352 (limb chains).
-constexpr uint32_t kColA = 0, kColDs = 256, kColDo = 320, kTmemColsTc = 512;
+// D_score x2 at 256, 288 (mse 16 | sgn 16); D_o regions x4 at 320 + 32 X
+// (two per softmax group; two value-limb chains of 16 columns each).
+constexpr uint32_t kColA = 0, kColDs = 256, kColDo = 320, kTmemCols = 512;
 
 // Instruction descriptor, kind::i8: s32 D, M = 128, N = 16.
-__host__ __device__ constexpr uint32_t idesc_i8(bool a_signed, bool a_mn_major) {
-  return (2u << 4) | ((a_signed ? 1u : 0u) << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
-         ((16u >> 3) << 17) | ((128u >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_i8(bool a_signed, bool a_mn_major, bool b_mn_major, bool b_signed) {
+  return (2u << 4) | ((a_signed ? 1u : 0u) << 7) | ((b_signed ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 template <int KB>
-struct TcSm {
+struct FSm {
   static constexpr int kRbk = kD * KB / 8;
-  static constexpr int kStageBytes = kTT * (kRbk + 16 + 48);       // kidx | ksign | vidx
+  static constexpr int kOffKs = kTT * kRbk;                        // sign rows within a stage
+  static constexpr int kOffVi = kOffKs + kTT * 16;                 // value index rows
+  static constexpr int kStageBytes = kOffVi + kTT * 48;
   static constexpr int kStageStride = ((kStageBytes + 1023) / 1024) * 1024;
-  static constexpr int kOffVh = kStages * kStageStride;            // 1024-aligned
-  static constexpr int kVhBytes = 2 * kTT * 128;                    // two limbs x 128 tokens x 128 B
-  static constexpr int kOffP = kOffVh + 2 * kVhBytes;               // 2 x [16 rows x 128 B]
-  static constexpr int kOffB = kOffP + 2 * 2048;                    // 2 items x (B1 | B2 | B3 | Bs)
-  static constexpr int kOffBar = kOffB + 2 * 4 * 2048;
-  static constexpr int kNumBars = 2 * kStages + 2 * 11 + 2;
-  static constexpr int kOffMisc = ((kOffBar + kNumBars * 8 + 15) / 16) * 16;
-  static constexpr int kOffRing = kOffMisc + 16;                    // [4 tiles][8]: corr[4], scale
-  static constexpr int kOffRed = kOffRing + 4 * 8 * 4;              // [2 groups][4 warps][16]
-  static constexpr int kOffRed2 = kOffRed + 2 * 4 * 16 * 4;         // [2 groups][4 warps][4]
-  static constexpr int kOffTab = kOffRed2 + 2 * 4 * 4 * 4;          // ka1 ka2 ka3 va1 va2 (4 words) + 2 scales
-  static constexpr int kBytes = kOffTab + 22 * 4 + 1024;
+  static constexpr int kOffVh = kStages * kStageStride;            // 2 buffers x 2 limbs x 16 KB
+  static constexpr int kVhBytes = 2 * kTT * 128;
+  static constexpr int kOffP = kOffVh + 2 * kVhBytes;              // 2 x [128 tokens][16 B]
+  static constexpr int kOffB = kOffP + 2 * 2048;                   // 2 segments x (B1 | B2 | B3 | Bs)
+  static constexpr int kOffQ = kOffB + 2 * 4 * 2048;               // qx, qr, sv: [4][128] floats each
+  static constexpr int kOffPP = kOffQ + 3 * kRows * kD * 4;        // [3][4][128] floats: matvec partials
+  static constexpr int kOffRed = kOffPP + 3 * kRows * kD * 4;      // [16][16] floats
+  static constexpr int kOffSeg = kOffRed + 16 * 16 * 4;            // [2][kSegFloats] per-segment constants
+  static constexpr int kOffNrm = kOffSeg + 2 * kSegFloats * 4;     // [2 groups][4 slots][3][128] norms
+  static constexpr int kOffRec = kOffNrm + 2 * 4 * 3 * kTT * 4;    // [8][16] words: tile records
+  static constexpr int kOffTab = kOffRec + 8 * 16 * 4;             // limb tables (20 words) + 2 scales
+  static constexpr int kOffBar = kOffTab + 32 * 4;
+  static constexpr int kNumBars = 2 * kStages + 7 * 2 + 4 + 4 + 2;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 64 + 1024;               // + alignment slack
 };
 
-struct TcDecodeArgs {
+static_assert(FSm<4>::kBytes <= 232448, "shared memory plan exceeds 227 KB");
+
+struct FusedArgs {
   DecodeArgs v;
-  int n_items;
+  int64_t T, Ts;       // tiles in all, tiles per stream
+  int V;               // virtual CTAs
+  int* counters;       // [streams] arrivals (zero at launch)
 };
 
-// int8 limbs of a codebook, c ~ scale (a1 + a2/128 + a3/128^2) with
-// scale = max|c| / 127, as byte tables (byte k of word k/4 = code k); t3 may
-// be null (two limbs). Computed in fp64 by one thread; every CTA derives the
-// same tables.
-__device__ void codebook_limbs(const float* c, int n, uint32_t* t1, uint32_t* t2, uint32_t* t3, float* scale) {
-  double m = 0.0;
-  for (int k = 0; k < n; ++k) m = fmax(m, fabs(static_cast<double>(__ldg(c + k))));
+// int8 limbs of the key codebook (three) and the value codebook (two),
+// c ~ scale (a1 + a2/128 + a3/128^2) with scale = max|c| / 127, as byte tables
+// (byte k of word k/4 = code k): tab[0..3] a1, [4..7] a2, [8..11] a3 (keys),
+// [12..15] a1, [16..19] a2 (values). One warp: lane k < nk takes key code k,
+// lane 16 + k value code k; fp64, so every CTA derives the same tables.
+__device__ void codebook_limbs_warp(const float* cK, int nk, const float* cV, uint32_t* tab, float* scales, int lane) {
+  const bool key = lane < 16, has = key ? lane < nk : lane < 24;
+  const int k = key ? lane : lane - 16;
+  const double c = has ? static_cast<double>(__ldg((key ? cK : cV) + k)) : 0.0;
+  double m = fabs(c);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));   // within each half
   const double sc = m > 0.0 ? m / 127.0 : 1.0;
-  for (int w = 0; w < 4; ++w) {
-    t1[w] = t2[w] = 0u;
-    if (t3) t3[w] = 0u;
-  }
-  auto put = [](uint32_t* t, int k, double v) {
-    t[k / 4] |= static_cast<uint32_t>(static_cast<uint8_t>(static_cast<int8_t>(v))) << (8 * (k % 4));
-  };
-  for (int k = 0; k < n; ++k) {
-    const double r0 = static_cast<double>(__ldg(c + k)) / sc;
+  if (lane < 20) tab[lane] = 0u;
+  __syncwarp();
+  if (has) {
+    unsigned char* tb = reinterpret_cast<unsigned char*>(tab) + (key ? 0 : 48);
+    const double r0 = c / sc;
     const double a1 = rint(r0);
     const double r1 = (r0 - a1) * 128.0;
     const double a2 = rint(r1);
-    put(t1, k, a1);
-    put(t2, k, a2);
-    if (t3) put(t3, k, rint((r1 - a2) * 128.0));
+    tb[k] = static_cast<unsigned char>(static_cast<int8_t>(a1));
+    tb[16 + k] = static_cast<unsigned char>(static_cast<int8_t>(a2));
+    if (key) tb[32 + k] = static_cast<unsigned char>(static_cast<int8_t>(rint((r1 - a2) * 128.0)));
   }
-  *scale = static_cast<float>(sc);
+  if (lane == 0) scales[0] = static_cast<float>(sc);
+  if (lane == 16) scales[1] = static_cast<float>(sc);
 }
 
 __device__ __forceinline__ bool wg_sync_or(int id, bool p) {
@@ -136,7 +159,16 @@ __device__ __forceinline__ bool wg_sync_or(int id, bool p) {
       : "memory");
   return r != 0;
 }
-__device__ __forceinline__ void wg_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+// One lane of the (converged) warp; the others get false.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
   uint32_t d;
@@ -204,62 +236,160 @@ __device__ __forceinline__ void limbs4(float x, int (&l)[4]) {
     x = (x - static_cast<float>(l[u])) * 128.f;
   }
 }
-// int32 accumulator -> float (exact: every accumulator here stays below 2^22,
-// at most 3 limb products of 128 terms with limbs <= 127 in magnitude).
-__device__ __forceinline__ float i2f(uint32_t x) { return static_cast<float>(static_cast<int32_t>(x)); }
-__device__ __forceinline__ float limb_sum4(const uint32_t* d) {
-  float v = i2f(d[3]);
-  v = fmaf(v, 1.f / 128.f, i2f(d[2]));
-  v = fmaf(v, 1.f / 128.f, i2f(d[1]));
-  return fmaf(v, 1.f / 128.f, i2f(d[0]));
-}
-__device__ __forceinline__ float limb_sum3(const uint32_t* d) {
-  return fmaf(fmaf(i2f(d[2]), 1.f / 128.f, i2f(d[1])), 1.f / 128.f, i2f(d[0]));
-}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t n) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// Shared-memory descriptor of an MN-major operand without swizzle whose
+// rows (one per K index) are 16 bytes: core matrices of 8 rows x 16 B, 128 B
+// apart along K.
+__device__ __forceinline__ uint64_t desc_mn_noswz(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;     // LBO
+  d |= static_cast<uint64_t>(128u >> 4) << 32;     // SBO
+  d |= static_cast<uint64_t>(1u) << 46;            // descriptor version for sm_100
+  return d;                                        // layout 0: no swizzle
+}
+
+// y[r][i] = sum_j M[i][j] x[r][j] for four rows (x, y: shared [4][128]) on
+// 384 threads: thread u takes output coordinate i = u % 128 and the input
+// coordinates of part u / 128 (44, 44, 40 of them, whole float4s), with all
+// of its row loads in flight; the three partial sums meet in pp [3][4][128].
+// Two barriers of the 384 threads (id 2).
+__device__ __forceinline__ void matvec4_split(const float* __restrict__ M, const float* x, float* y, float* pp, int u) {
+  const int i = u & 127, part = u >> 7;
+  const int j4_0 = part * 11, n4 = part == 2 ? 10 : 11;
+  const float4* row = reinterpret_cast<const float4*>(M + int64_t(i) * kD) + j4_0;
+  float4 mv[11];
+#pragma unroll
+  for (int k = 0; k < 11; ++k) mv[k] = k < n4 ? __ldg(row + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+  float acc[kRows] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < 11; ++k) {
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      const float4 xv = reinterpret_cast<const float4*>(x + r * kD)[j4_0 + (k < n4 ? k : 0)];
+      acc[r] = fmaf(mv[k].x, xv.x, fmaf(mv[k].y, xv.y, fmaf(mv[k].z, xv.z, fmaf(mv[k].w, xv.w, acc[r]))));
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) pp[(part * kRows + r) * kD + i] = acc[r];
+  named_sync(2, 384);
+  if (u < 128) {
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) y[r * kD + i] = pp[r * kD + i] + pp[(kRows + r) * kD + i] + pp[(2 * kRows + r) * kD + i];
+  }
+  named_sync(2, 384);
+}
+
+// Work partition: all (stream, tile) pairs in stream order, cut into V equal
+// contiguous ranges ("virtual CTAs", V >= grid); physical CTA c takes v = c,
+// c + grid, ... A range splits at stream ends into segments; the segment of
+// virtual CTA v in stream s owns partial record v + s (the pair is unique
+// because both the ranges and the streams are ordered).
+struct Part {
+  int64_t T;      // tiles in all
+  int64_t Ts;     // tiles per stream
+  int V;          // virtual CTAs
+};
+__device__ __forceinline__ int64_t vstart(const Part& p, int64_t v) { return (v * p.T) / p.V; }
+// Virtual CTA holding global tile g.
+__device__ __forceinline__ int64_t vof(const Part& p, int64_t g) {
+  int64_t v = (g * p.V) / p.T;
+  while (v > 0 && vstart(p, v) > g) --v;
+  while (v + 1 < p.V && vstart(p, v + 1) <= g) ++v;
+  return v;
+}
+
+struct Seg {
+  int64_t v, s;        // virtual CTA, stream
+  int64_t t0, t1;      // tiles [t0, t1) of the stream
+  int idx;             // segment number within this CTA
+};
+// Segments of this CTA, in order (every role walks the same sequence).
+struct SegIter {
+  Part p;
+  int64_t v, g, g1;
+  int idx;
+  __device__ SegIter(const Part& pp) : p(pp), v(blockIdx.x), g(0), g1(0), idx(0) {
+    if (v < p.V) {
+      g = vstart(p, v);
+      g1 = vstart(p, v + 1);
+    }
+  }
+  __device__ bool next(Seg& sg) {
+    while (v < p.V && g >= g1) {
+      v += gridDim.x;
+      if (v < p.V) {
+        g = vstart(p, v);
+        g1 = vstart(p, v + 1);
+      }
+    }
+    if (v >= p.V) return false;
+    const int64_t s = g / p.Ts;
+    const int64_t ge = min(g1, (s + 1) * p.Ts);
+    sg.v = v;
+    sg.s = s;
+    sg.t0 = g - s * p.Ts;
+    sg.t1 = ge - s * p.Ts;
+    sg.idx = idx++;
+    g = ge;
+    return true;
+  }
+};
+
 template <int KB>
-__global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A) {
-  using Sm = TcSm<KB>;
+__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) {
+  using Sm = FSm<KB>;
   constexpr int kRbk = Sm::kRbk;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const DecodeArgs& a = A.v;
+  const DecodeShape& sh = a.sh;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Sm::kOffBar);
-  uint64_t* st_full = bars;                       // [3]
-  uint64_t* st_empty = bars + kStages;            // [3]
-  uint64_t* a_full = bars + 2 * kStages;          // [2]
-  uint64_t* a_free = a_full + 2;                  // [2] (aliased below)
-  uint64_t* s_full = a_free + 2;                  // [2]
-  uint64_t* ds_free = s_full + 2;                 // [2]
-  uint64_t* vh_full = ds_free + 2;                // [2]
-  uint64_t* vh_free = vh_full + 2;                // [2] (aliased below)
-  uint64_t* p_full = vh_free + 2;                 // [2]
-  uint64_t* p_free = p_full + 2;                  // [2] (aliased below)
-  uint64_t* pv_full = p_free + 2;                 // [2]
-  uint64_t* do_free = pv_full + 2;                // [2]
-  uint64_t* b_full = do_free + 2;                 // [2] per item parity
-  uint64_t* drain = b_full + 2;                   // [2] score issuer, PV issuer
-  // One completion event each: the score MMAs of a tile free its key operands
-  // and fill its score columns; the PV MMAs free the value operands and the
-  // weight tile and fill the value columns.
-  a_free = s_full;
-  vh_free = pv_full;
-  p_free = pv_full;
+  uint64_t* st_full = bars;                       // [kStages] loader (tx)
+  uint64_t* st_empty = bars + kStages;            // [kStages] 4 key + 4 value warps
+  uint64_t* a_full = bars + 2 * kStages;          // [2] key warps
+  uint64_t* s_full = a_full + 2;                  // [2] score commit (also frees the A operand)
+  uint64_t* ds_free = s_full + 2;                 // [2] softmax warps read the score columns
+  uint64_t* vh_full = ds_free + 2;                // [2] value warps
+  uint64_t* p_full = vh_full + 2;                 // [2] softmax warps
+  uint64_t* pv_full = p_full + 2;                 // [2] PV commit (frees the value operand and P)
+  uint64_t* bt_full = pv_full + 2;                // [2] per segment parity: the prologue's 8 warps
+  uint64_t* reg_done = bt_full + 2;               // [4] PV commit when a TMEM value region closes
+  uint64_t* reg_free = reg_done + 4;              // [4] value warps folded the region
+  uint64_t* drain = reg_free + 4;                 // [2] score issuer, PV issuer
+  uint64_t* a_free = s_full;
+  uint64_t* vh_free = pv_full;
+  uint64_t* p_free = pv_full;
+
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Sm::kOffMisc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + Sm::kOffMisc + 4);
-  float* ring = reinterpret_cast<float*>(sm + Sm::kOffRing);          // [4][8]
-  float* red = reinterpret_cast<float*>(sm + Sm::kOffRed);            // [4 warps][16]
-  float* red2 = reinterpret_cast<float*>(sm + Sm::kOffRed2);          // [4 warps][4]
-  uint32_t* tab = reinterpret_cast<uint32_t*>(sm + Sm::kOffTab);      // ka1 ka2 ka3 va1 va2 (4 words each)
-  float* cb_scale = reinterpret_cast<float*>(sm + Sm::kOffTab + 20 * 4);   // key, value codebook scales
+  int* merge_s = reinterpret_cast<int*>(sm + Sm::kOffMisc + 8);
+  float* qx = reinterpret_cast<float*>(sm + Sm::kOffQ);             // [4][128] RoPE'd q; merged rows
+  float* qr = qx + kRows * kD;                                      // [4][128] q_rot
+  float* sv = qr + kRows * kD;                                      // [4][128] s
+  float* red = reinterpret_cast<float*>(sm + Sm::kOffRed);          // [16][16]
+  float* pp = reinterpret_cast<float*>(sm + Sm::kOffPP);            // [3][4][128] partial sums
+  float* segc = reinterpret_cast<float*>(sm + Sm::kOffSeg);         // [2][kSegFloats] per-segment constants
+  uint32_t* recs = reinterpret_cast<uint32_t*>(sm + Sm::kOffRec);   // [8][16] tile records
+  uint32_t* tab = reinterpret_cast<uint32_t*>(sm + Sm::kOffTab);    // ka1 ka2 ka3 va1 va2 (4 words each)
+  float* cb_scale = reinterpret_cast<float*>(sm + Sm::kOffTab + 20 * 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const DecodeShape& sh = a.sh;
+  const Part part{A.T, A.Ts, A.V};
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -268,35 +398,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&a_full[b], 4);
-      mbar_init(&a_free[b], 1);
       mbar_init(&s_full[b], 1);
       mbar_init(&ds_free[b], 4);
       mbar_init(&vh_full[b], 4);
-      mbar_init(&vh_free[b], 1);
       mbar_init(&p_full[b], 4);
-      mbar_init(&p_free[b], 1);
       mbar_init(&pv_full[b], 1);
-      mbar_init(&do_free[b], 4);
-      mbar_init(&b_full[b], 4);
+      mbar_init(&bt_full[b], 8);
+      mbar_init(&drain[b], 1);
     }
-    mbar_init(&drain[0], 1);
-    mbar_init(&drain[1], 1);
+    for (int x = 0; x < 4; ++x) {
+      mbar_init(&reg_done[x], 1);
+      mbar_init(&reg_free[x], 4);
+    }
     *abort_s = 0;
-    for (int k = 0; k < 4; ++k) reinterpret_cast<int*>(sm + Sm::kOffRing)[k * 8 + 5] = -1;
+    for (int k = 0; k < 8; ++k) recs[k * 16] = 0xFFFFFFFFu;
     mbar_fence_init();
   }
-  if (tid == 32) {
-    codebook_limbs(a.cK, 1 << sh.kbits, tab, tab + 4, tab + 8, &cb_scale[0]);
-    codebook_limbs(a.cV, 8, tab + 12, tab + 16, nullptr, &cb_scale[1]);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_base_s, kTmemColsTc);
+  if (warp == 3) codebook_limbs_warp(a.cK, 1 << sh.kbits, a.cV, tab, cb_scale, lane);
+  if (warp == kWScore) {
+    tmem_alloc(tmem_base_s, kTmemCols);
     tmem_relinquish();
-  }
-  // Rows 12-15 of both weight tiles stay zero (3 limbs x 4 rows are used).
-  for (int e = tid; e < 2 * 512 / 16; e += kThreadsTc) {
-    const int b = e / 32, o = e % 32;
-    reinterpret_cast<uint4*>(sm + Sm::kOffP + b * 2048 + 1536)[o] = make_uint4(0u, 0u, 0u, 0u);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -308,40 +429,28 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
     if (a.d_status) atomicOr(a.d_status, TQ_DEV_TIMEOUT);
   };
   const float k_scale = cb_scale[0], v_scale = cb_scale[1];
+  const int G = sh.hq / sh.hkv;
 
-  // Item sequence (identical in every role): items blockIdx.x, +gridDim.x, ...
-  // item -> (unit, split); tiles of 128 tokens inside the split.
-  auto item_tiles = [&](int item, int64_t& t_begin, int64_t& t_end) -> int {
-    const int split = item % sh.n_splits;
-    t_begin = int64_t(split) * sh.chunk;
-    t_end = (t_begin + sh.chunk < sh.n_ctx) ? t_begin + sh.chunk : sh.n_ctx;
-    return static_cast<int>((t_end - t_begin + kTT - 1) / kTT);
-  };
-  auto item_row0 = [&](int item) -> int64_t {
-    const int64_t unit = item / sh.n_splits;       // row_blocks == 1 for this kernel
-    return unit * sh.ctx_stride;
-  };
-
-  if (warp == 0) {
+  if (warp == kWLoader) {
     // ------------------------------------------------------------- loader
     if (lane == 0) {
       int j = 0;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < A.n_items; item += gridDim.x) {
-        int64_t tb, te;
-        const int nt_tiles = item_tiles(item, tb, te);
-        const int64_t row0 = item_row0(item);
-        for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
+      SegIter it(part);
+      Seg sg;
+      while (ok && it.next(sg)) {
+        const int64_t row0 = sg.s * sh.ctx_stride;
+        for (int64_t tt = sg.t0; tt < sg.t1; ++tt, ++j) {
           const int s = j % kStages;
           if (*abort_s || !mbar_wait(&st_empty[s], ((j / kStages) & 1) ^ 1)) { ok = false; break; }
-          const int64_t t0 = tb + int64_t(tj) * kTT;
-          const int nt = static_cast<int>((te - t0 < kTT) ? te - t0 : kTT);
+          const int64_t t0 = tt * kTT;
+          const int nt = static_cast<int>((sh.n_ctx - t0 < kTT ? sh.n_ctx - t0 : int64_t(kTT)));
           const uint32_t bk = nt * kRbk, bs = nt * 16, bv = nt * 48;
           mbar_expect_tx(&st_full[s], bk + bs + bv);
           unsigned char* st = sm + s * Sm::kStageStride;
           bulk_g2s(st, a.kidx + (row0 + t0) * kRbk, bk, &st_full[s]);
-          bulk_g2s(st + kTT * kRbk, a.ksign + (row0 + t0) * 4, bs, &st_full[s]);
-          bulk_g2s(st + kTT * (kRbk + 16), a.vidx + (row0 + t0) * 48, bv, &st_full[s]);
+          bulk_g2s(st + Sm::kOffKs, a.ksign + (row0 + t0) * 4, bs, &st_full[s]);
+          bulk_g2s(st + Sm::kOffVi, a.vidx + (row0 + t0) * 48, bv, &st_full[s]);
         }
       }
       if (!ok && !*abort_s) fail();
@@ -351,70 +460,101 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         mbar_wait(&st_full[jj % kStages], (jj / kStages) & 1);
       }
     }
-  } else if (warp == 1 || warp == 14) {
-    // ------------------------------------------ MMA issuers (one thread each)
-    // warp 1 issues the score MMAs, warp 14 the PV MMAs, so the issue
-    // latencies of the two chains overlap.
-    if (lane == 0) {
-      const uint32_t id_mse = idesc_i8(true, false), id_sgn = idesc_i8(false, false), id_v = idesc_i8(true, true);
-      const uint64_t p_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffP));
-      const uint64_t b_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffB));
-      const uint64_t vh_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffVh));
-      int j = 0, s_k = 0;
-      bool ok = true;
-      for (int item = blockIdx.x; ok && item < A.n_items; item += gridDim.x, ++s_k) {
-        int64_t tb, te;
-        const int nt_tiles = item_tiles(item, tb, te);
-        for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
-          const int b = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          if (*abort_s) { ok = false; break; }
-          if (warp == 1) {
-            const int ib = s_k & 1;
-            if (!mbar_wait(&b_full[ib], (s_k >> 1) & 1) || !mbar_wait(&a_full[b], ph) ||
-                !mbar_wait(&ds_free[b], ph ^ 1)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t d = tmem + kColDs + b * 32;
-            const uint32_t a0 = tmem + kColA + b * 128;
-            // a1, a2, a3 against B1, B2, B3 (limb-shifted q) into the MSE
-            // columns, the sign chunk into its own columns.
-            const uint64_t bs = b_desc0 + (((ib * 4 + 3) * 2048) >> 4);
+  } else if (warp == kWScore || warp == kWPv) {
+    // ------------------------------------------ MMA issuers (one warp each)
+    // The whole warp runs the loop (descriptor arithmetic stays warp-uniform)
+    // and one elected lane issues each MMA: issuing from a divergent
+    // single-lane branch costs several times more per MMA.
+    const bool leader = elect_one();
+    const uint32_t id_mse = idesc_i8(true, false, false, true), id_sgn = idesc_i8(false, false, false, true);
+    const uint32_t id_v = idesc_i8(true, true, true, false);
+    const uint64_t b_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffB));
+    const uint64_t vh_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffVh));
+    const uint64_t p_desc0 = desc_mn_noswz(smem_u32(sm + Sm::kOffP));
+    int j = 0;
+    bool ok = true;
+    // PV: TMEM region in use per softmax group (2 g + bit g of pcur) and the
+    // closes per region (byte X of pcl), kept in registers.
+    uint32_t pcur = 0u, pcl = 0u;
+    SegIter it(part);
+    Seg sg;
+    while (ok && it.next(sg)) {
+      const int ib = sg.idx & 1;
+      const int nt_tiles = static_cast<int>(sg.t1 - sg.t0);
+      if (warp == kWScore &&
+          !__all_sync(0xffffffffu, mbar_wait(&bt_full[ib], (sg.idx >> 1) & 1))) { ok = false; break; }
+      for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
+        const int b = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (__any_sync(0xffffffffu, *abort_s != 0)) { ok = false; break; }
+        if (warp == kWScore) {
+          const bool w = mbar_wait(&a_full[b], ph) && mbar_wait(&ds_free[b], ph ^ 1);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + kColDs + b * 32;
+          const uint32_t a0 = tmem + kColA + b * 128;
+          // a1, a2, a3 against B1, B2, B3 (limb-shifted q) into the MSE
+          // columns, the sign chunk into its own columns.
+          const uint64_t bs = b_desc0 + (((ib * 4 + 3) * 2048) >> 4);
 #pragma unroll
-            for (int step = 0; step < 12; ++step) {
-              const int ch = step >> 2, k = step & 3;
-              const uint64_t bq = b_desc0 + (((ib * 4 + ch) * 2048) >> 4);
-              umma_i8_ts(d, a0 + ch * 32 + k * 8, bq + ((k * 32) >> 4), id_mse, step != 0);
-              if (step < 4) umma_i8_ts(d + 16, a0 + 96 + k * 8, bs + ((k * 32) >> 4), id_sgn, k != 0);
-            }
-            umma_commit(&s_full[b]);
-          } else {
-            if (!mbar_wait(&vh_full[b], ph) || !mbar_wait(&p_full[b], ph) || !mbar_wait(&do_free[b], ph ^ 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t d = tmem + kColDo + b * 32;
-            const uint64_t pb = p_desc0 + ((b * 2048) >> 4);
+          for (int step = 0; step < 12; ++step) {
+            const int ch = step >> 2, k = step & 3;
+            const uint64_t bq = b_desc0 + (((ib * 4 + ch) * 2048) >> 4);
+            if (leader) umma_i8_ts(d, a0 + ch * 32 + k * 8, bq + ((k * 32) >> 4), id_mse, step != 0);
+            if (step < 4 && leader) umma_i8_ts(d + 16, a0 + 96 + k * 8, bs + ((k * 32) >> 4), id_sgn, k != 0);
+          }
+          if (leader) umma_commit(&s_full[b]);
+        } else {
+          const bool w = mbar_wait(&vh_full[b], ph) && mbar_wait(&p_full[b], ph);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          tc_fence_after();
+          const bool flip = recs[(j & 7) * 16 + 1] != 0u;
+          const int g = tj & 1;                     // softmax group of the tile
+          bool fresh = tj == g;                     // the group's first tile of the segment
+          if (flip && !fresh) {
+            // The group's running maximum moved: close its region (its MMAs
+            // so far are tracked by this commit) and continue in its other one.
+            const int Xc = 2 * g + static_cast<int>((pcur >> g) & 1u);
+            if (leader) umma_commit(&reg_done[Xc]);
+            pcl += 1u << (8 * Xc);
+            pcur ^= 1u << g;
+            fresh = true;
+          }
+          const int X = 2 * g + static_cast<int>((pcur >> g) & 1u);
+          const uint32_t nclose = (pcl >> (8 * X)) & 0xFFu;
+          if (fresh && nclose > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(&reg_free[X], (nclose - 1) & 1))) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + kColDo + X * 32;
+          const uint64_t pb = p_desc0 + ((b * 2048) >> 4);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {             // 32 tokens per step = 4 atoms of 8 tokens
+          for (int k = 0; k < 4; ++k) {             // 32 tokens per step = 4 atoms of 8 tokens
 #pragma unroll
-              for (int limb = 0; limb < 2; ++limb) {  // the two limb chains alternate
-                const uint64_t ad = vh_desc0 + ((b * Sm::kVhBytes + limb * kTT * 128 + k * 4096) >> 4);
-                umma_i8_ss(d + limb * 16, ad, pb + ((k * 32) >> 4), id_v, k != 0);
-              }
+            for (int limb = 0; limb < 2; ++limb) {  // the two limb chains alternate
+              const uint64_t ad = vh_desc0 + ((b * Sm::kVhBytes + limb * kTT * 128 + k * 4096) >> 4);
+              if (leader) umma_i8_ss(d + limb * 16, ad, pb + ((k * 512) >> 4), id_v, !(fresh && k == 0));
             }
-            umma_commit(&pv_full[b]);
+          }
+          if (leader) umma_commit(&pv_full[b]);
+          if (tj >= nt_tiles - 2) {
+            // The group's last tile of the segment: close its region; its next
+            // segment starts in the other one.
+            if (leader) umma_commit(&reg_done[X]);
+            pcl += 1u << (8 * X);
+            pcur ^= 1u << g;
           }
         }
+        __syncwarp();
       }
-      if (!ok && !*abort_s) fail();
-      // Every MMA this thread issued completes before TMEM is released.
-      umma_commit(&drain[warp == 1 ? 0 : 1]);
-      mbar_wait(&drain[warp == 1 ? 0 : 1], 0);
     }
-  } else if (warp < 6) {
+    if (!ok && leader && !*abort_s) fail();
+    // Every MMA this warp issued completes before TMEM is released.
+    if (leader) umma_commit(&drain[warp == kWScore ? 0 : 1]);
+    __syncwarp();
+    mbar_wait(&drain[warp == kWScore ? 0 : 1], 0);
+  } else if (warp >= kWKey0 && warp < kWKey0 + 4) {
     // ------------------------------------------------- key operands (TMEM)
-    const int q = warp & 3;                       // lane quadrant (warps 2..5 -> 2,3,0,1)
+    const int q = warp & 3;                       // lane quadrant
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int row = q * 32 + lane;                // token = TMEM lane this thread writes
     uint32_t k1[4], k2[4], k3[4];
@@ -426,9 +566,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
     }
     int j = 0;
     bool stop = false;
-    for (int item = blockIdx.x; !stop && item < A.n_items; item += gridDim.x) {
-      int64_t tb, te;
-      const int nt_tiles = item_tiles(item, tb, te);
+    SegIter it(part);
+    Seg sg;
+    while (!stop && it.next(sg)) {
+      const int nt_tiles = static_cast<int>(sg.t1 - sg.t0);
       for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
         const int s = j % kStages;
         const int b = j & 1;
@@ -438,16 +579,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
           break;
         }
         const unsigned char* st = sm + s * Sm::kStageStride;
-        uint32_t w[kRbk / 4 + 1];
-#pragma unroll
-        for (int u = 0; u < kRbk / 16; ++u) {
-          const uint4 x = reinterpret_cast<const uint4*>(st + row * kRbk)[u];
-          w[4 * u] = x.x; w[4 * u + 1] = x.y; w[4 * u + 2] = x.z; w[4 * u + 3] = x.w;
-        }
-        w[kRbk / 4] = 0u;
-        const uint4 sg = reinterpret_cast<const uint4*>(st + kTT * kRbk + row * 16)[0];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&st_empty[s]);
+        // The row's code words stay in shared memory until the limbs are
+        // built (read KB words per 32 coordinates); the stage is released
+        // after the last read.
+        const uint32_t* wrow = reinterpret_cast<const uint32_t*>(st + row * kRbk);
+        const uint4 sg4 = reinterpret_cast<const uint4*>(st + Sm::kOffKs + row * 16)[0];
         if (!__all_sync(0xffffffffu, mbar_wait(&a_free[b], ((j >> 1) & 1) ^ 1))) {
           if (lane == 0) fail();
           stop = true;
@@ -455,14 +591,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         }
         tc_fence_after();
         const uint32_t acol = lane_addr + kColA + b * 128;
-        // 32 coordinates per iteration (KB words of codes, w[0..KB-1]; the
-        // words shift down after each one): nibble selectors, then the three
-        // limbs of each coordinate by byte permutes into 8 TMEM columns per limb.
+        // 32 coordinates per iteration (KB words of codes): nibble selectors,
+        // then the three limbs of each coordinate by byte permutes into 8 TMEM
+        // columns per limb.
 #pragma unroll 1
         for (int qq = 0; qq < 4; ++qq) {
           uint32_t xq[KB + 1];
 #pragma unroll
-          for (int u = 0; u < KB; ++u) xq[u] = w[u];
+          for (int u = 0; u < KB; ++u) xq[u] = wrow[qq * KB + u];
           xq[KB] = 0u;
           uint32_t nib[4];
 #pragma unroll
@@ -490,16 +626,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
             }
             tmem_st8(acol + limb * 32 + qq * 8, v8);
           }
-#pragma unroll
-          for (int u = 0; u + KB < kRbk / 4 + 1; ++u) w[u] = w[u + KB];
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&st_empty[s]);
         uint32_t v[32];
         // Sign chunk: column 4 m + u = sign word u AND (0x01010101 << m).
-        const uint32_t sw[4] = {sg.x, sg.y, sg.z, sg.w};
+        const uint32_t swd[4] = {sg4.x, sg4.y, sg4.z, sg4.w};
 #pragma unroll
         for (int m = 0; m < 8; ++m)
 #pragma unroll
-          for (int u = 0; u < 4; ++u) v[4 * m + u] = sw[u] & (0x01010101u << m);
+          for (int u = 0; u < 4; ++u) v[4 * m + u] = swd[u] & (0x01010101u << m);
         tmem_st32(acol + 96, v);
         tmem_st_wait();
         tc_fence_before();
@@ -507,393 +643,601 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
         if (lane == 0) mbar_arrive(&a_full[b]);
       }
     }
-  } else if (warp < 10) {
-    // ------------------------------- value operands (smem), value epilogue
-    const int row = tid - 192;                    // token within the tile (operands)
-    const int q = warp & 3;                       // lane quadrant (warps 6..9 -> 2,3,0,1)
-    const int crd = q * 32 + lane;                // coordinate = TMEM lane (epilogue)
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t v1t[2] = {tab[12], tab[13]}, v2t[2] = {tab[16], tab[17]};
-    int j = 0;
-    bool stop = false;
-    float acc[2][kRowsTc];                        // even / odd tiles of the item
-    // Value epilogue of tile jj (this thread = coordinate crd): wait for its
-    // PV product, then for ring slot jj % 4 to carry tag jj (the softmax warps
-    // write the tile's corrections and scale, fence, then the tag; the slot is
-    // rewritten only after PV(jj + 2), which needs this epilogue's do_free).
-    auto value_epilogue = [&](int jj) -> bool {
-      const int b2 = jj & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&pv_full[b2], (jj >> 1) & 1))) return false;
-      tc_fence_after();
-      uint32_t d[32];
-      tmem_ld32(lane_addr + kColDo + b2 * 32, d);
-      volatile int* tag = reinterpret_cast<volatile int*>(ring + (jj & 3) * 8 + 5);
-      bool tag_ok = *tag == jj;
-      if (!tag_ok) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!(tag_ok = (*tag == jj)) && globaltimer_ns() - t0 < 2000000000ull) {
-        }
-      }
-      __threadfence_block();
-      const float4 c4 = reinterpret_cast<const float4*>(ring + (jj & 3) * 8)[0];
-      const float spv = ring[(jj & 3) * 8 + 4] * v_scale;
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&do_free[b2]);
-      if (!__all_sync(0xffffffffu, tag_ok)) return false;
-      const float corr[kRowsTc] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) {
-        // column (r, weight limb l) = 3 r + l in each value-limb chain
-        const float hi = limb_sum3(d + 3 * r), lo = limb_sum3(d + 16 + 3 * r);
-        acc[b2][r] = fmaf(acc[b2][r], corr[r], spv * fmaf(lo, 1.f / 128.f, hi));
-      }
-      return true;
-    };
-    for (int item = blockIdx.x; !stop && item < A.n_items; item += gridDim.x) {
-      int64_t tb, te;
-      const int nt_tiles = item_tiles(item, tb, te);
-#pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) acc[0][r] = acc[1][r] = 0.f;
-      for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
-        const int s = j % kStages;
-        const int b = j & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&st_full[s], (j / kStages) & 1))) {
-          if (lane == 0) fail();
-          stop = true;
-          break;
-        }
-        const unsigned char* st = sm + s * Sm::kStageStride;
-        uint32_t w[13];
-#pragma unroll
-        for (int u = 0; u < 3; ++u) {
-          const uint4 x = reinterpret_cast<const uint4*>(st + kTT * (kRbk + 16) + row * 48)[u];
-          w[4 * u] = x.x; w[4 * u + 1] = x.y; w[4 * u + 2] = x.z; w[4 * u + 3] = x.w;
-        }
-        w[12] = 0u;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&st_empty[s]);
-        if (!__all_sync(0xffffffffu, mbar_wait(&vh_free[b], ((j >> 1) & 1) ^ 1))) {
-          if (lane == 0) fail();
-          stop = true;
-          break;
-        }
-        unsigned char* vh = sm + Sm::kOffVh + b * Sm::kVhBytes;
-        // Row `row` (token) of each limb tile: 128 coordinate bytes, M-major,
-        // 8-token atoms of 1024 bytes. 32 coordinates (12 code bytes, w[0..2])
-        // per iteration; the words shift down after each one.
-        const int atom = row >> 3, r8 = row & 7;
-#pragma unroll 1
-        for (int c2 = 0; c2 < 4; ++c2) {
-          const uint32_t x4[4] = {w[0], w[1], w[2], 0u};
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {          // 16 coordinates = 6 bytes of codes
-            uint32_t o1[4], o2[4];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {           // 8 codes per half
-              const int g = 2 * cc + h;
-              const int off = 3 * g, wi = off >> 2, shf = 8 * (off & 3);
-              const uint32_t x = shf == 0 ? x4[wi] : __funnelshift_r(x4[wi], x4[wi + 1], shf);
-              const uint32_t nb = nibbles3(x);
-              o1[2 * h] = prmt(v1t[0], v1t[1], nb);
-              o1[2 * h + 1] = prmt(v1t[0], v1t[1], nb >> 16);
-              o2[2 * h] = prmt(v2t[0], v2t[1], nb);
-              o2[2 * h + 1] = prmt(v2t[0], v2t[1], nb >> 16);
-            }
-            const int c16 = 2 * c2 + cc;
-            const uint32_t off = atom * 1024 + r8 * 128 + ((c16 ^ r8) << 4);
-            *reinterpret_cast<uint4*>(vh + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-            *reinterpret_cast<uint4*>(vh + kTT * 128 + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
-          }
-#pragma unroll
-          for (int u = 0; u < 9; ++u) w[u] = w[u + 3];
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&vh_full[b]);
-        // Fold the previous tile of this item (its PV product is under way or done).
-        if (tj >= 1 && !value_epilogue(j - 1)) {
-          if (lane == 0) fail();
-          stop = true;
-          break;
-        }
-      }
-      if (stop) break;
-      if (!value_epilogue(j - 1)) {
-        if (lane == 0) fail();
-        break;
-      }
-      // Rotated-value partials of the item's even and odd tiles (records
-      // 2 split + parity; m and l come from the softmax warps).
-      const int64_t unit = item / sh.n_splits;
-      const int split = item % sh.n_splits;
-      const int kv = static_cast<int>(unit % sh.hkv), bb = static_cast<int>(unit / sh.hkv);
-      const int G = sh.hq / sh.hkv;
-#pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) {
-        const int64_t qr = (int64_t(bb) * sh.hq + kv * G + r / sh.nq) * sh.nq + r % sh.nq;
-        float* pr = a.part + (qr * sh.n_parts + 2 * split) * (kD + 2) + crd;
-        pr[0] = acc[0][r];
-        pr[kD + 2] = acc[1][r];
-      }
-    }
-  } else if (warp < 14) {
-    // ------------------- scores and softmax: even and odd tiles kept apart
-    constexpr int wg = 0;
-    const int cw = warp - 10;                     // warp within the group
-    const int q = warp & 3;                       // lane quadrant (2,3,0,1 per group)
-    const int lrow = q * 32 + lane;               // TMEM lane = token
-    const int bar_id = 1 + wg;
-    float* gred = red + wg * 64;
-    float* gred2 = red2 + wg * 16;
+  } else if (warp >= kWVal0) {
+    // ------------------------------------------ value warps and softmax warps
+    // The value group and both softmax groups share the per-segment prologue
+    // and the combine's arrival (384 threads on barrier 2); then each runs its
+    // own per-tile loop. Softmax group g takes the segment's tiles tj with
+    // tj % 2 == g and keeps its own running maxima, sums and TMEM regions
+    // (2g, 2g + 1), so the two groups' per-tile chains overlap.
+    const bool is_val = warp < kWSoft0;
+    const int sgrp = is_val ? -1 : (warp - kWSoft0) >> 2;   // softmax group
+    const int sbar = sgrp == 0 ? 1 : 4;                       // its named barrier (128 threads)
+    const int u = tid - kWVal0 * 32;              // 0..383; the prologue's work is on u < 256
+    const int q = warp & 3;                       // lane quadrant
+    const int lrow = q * 32 + lane;               // token (TMEM lane) / coordinate
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const float alpha = static_cast<float>(dev::kSqrtHalfPi / kD);
     constexpr float kLog2e = 1.4426950408889634f;
-    constexpr float kMagic = 12582912.f;          // 1.5 * 2^23: x + kMagic rounds x to an integer
-    // Byte offsets of this token's column in the 12 used rows of a weight tile.
-    uint32_t poff[12];
-#pragma unroll
-    for (int n = 0; n < 12; ++n) poff[n] = sw_byte(n, lrow);
-    int j = 0, item_idx = 0;
+    const uint32_t v1t[2] = {tab[12], tab[13]}, v2t[2] = {tab[16], tab[17]};
+    int j = 0;                                    // CTA-local tile counter
     bool stop = false;
-    for (int item = blockIdx.x; item < A.n_items && !stop; item += gridDim.x, ++item_idx) {
-      int64_t tb, te;
-      const int nt_tiles = item_tiles(item, tb, te);
-      const int64_t unit = item / sh.n_splits;
-      const int split = item % sh.n_splits;
-      const int kv = static_cast<int>(unit % sh.hkv), bb = static_cast<int>(unit / sh.hkv);
-      const int G = sh.hq / sh.hkv;
-      const int64_t row0 = item_row0(item);
-      int64_t qrow[kRowsTc];
-#pragma unroll
-      for (int r = 0; r < kRowsTc; ++r)
-        qrow[r] = (int64_t(bb) * sh.hq + kv * G + r / sh.nq) * sh.nq + r % sh.nq;
-      // ---- item prologue: row scales, the item's largest ||v||; group 0
-      // also writes the item's B tiles.
-      const int ib = item_idx & 1;
-      float sq[kRowsTc], ss[kRowsTc], ssum[kRowsTc], sp;
+    // value warps: TMEM region bookkeeping (mirrors the PV issuer)
+    int vcur[2] = {0, 0};
+    int closes[4] = {0, 0, 0, 0};
+    SegIter it(part);
+    Seg sg;
+    while (it.next(sg)) {
+      const int ib = sg.idx & 1;
+      const int nt_tiles = static_cast<int>(sg.t1 - sg.t0);
+      const int64_t bkv = sg.s;                   // stream = b * hkv + kv
+      const int kv = static_cast<int>(bkv % sh.hkv), bb = static_cast<int>(bkv / sh.hkv);
+      const int64_t row0 = bkv * sh.ctx_stride;
+      const int64_t te = (sg.t1 * kTT < sh.n_ctx ? sg.t1 * kTT : sh.n_ctx);
+      const int64_t rec_idx = sg.v + sg.s;
+      const int j0 = j;
+      auto qrow = [&](int r) -> int64_t { return int64_t(bb) * sh.hq + kv * G + r; };   // nq == 1
+      float* segk = segc + ib * kSegFloats;
+      // Softmax group: norms of its k-th tile (tile 2k + g) go into ring slot
+      // k % 4, three tiles ahead, by cp.async (one commit group per tile).
+      float* nring = reinterpret_cast<float*>(sm + Sm::kOffNrm) + (sgrp < 0 ? 0 : sgrp) * (4 * 3 * kTT);
+      auto norm_fetch = [&](int k) {
+        const int tj = 2 * k + sgrp;
+        if (tj < nt_tiles) {
+          const int64_t t = (sg.t0 + tj) * kTT + lrow;
+          const bool ok = t < te;
+          const int64_t off = row0 + (ok ? t : 0);
+          const uint32_t n = ok ? 4u : 0u;
+          float* slot = nring + (k & 3) * (3 * kTT);
+          cp_async4(smem_u32(slot + lrow), a.knorm + off, n);
+          cp_async4(smem_u32(slot + kTT + lrow), a.krnorm + off, n);
+          cp_async4(smem_u32(slot + 2 * kTT + lrow), a.vnorm + off, n);
+        }
+        cp_async_commit();
+      };
+      if (!is_val) {
+        norm_fetch(0);
+        norm_fetch(1);
+        norm_fetch(2);
+      }
+      // ---------------- prologue: q_rot = Pi_K RoPE(q), s = S q_rot, B tiles
       {
-        const int crd = lrow;                     // thread = coordinate here
-        const float jscale = __uint_as_float(static_cast<uint32_t>(127 - (crd & 7)) << 23);   // 2^-(i mod 8)
-        float qv[kRowsTc], sv[kRowsTc], loc[13];
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          qv[r] = a.qs[qrow[r] * 2 * kD + crd];
-          sv[r] = a.qs[qrow[r] * 2 * kD + kD + crd];
-          loc[r] = fabsf(qv[r]);
-          loc[4 + r] = fabsf(sv[r]) * jscale;
-          loc[8 + r] = sv[r];
+        const bool work = u < 256;
+        const bool rope = a.q_pos != nullptr && a.rope_base > 0.0;
+        if (work) {
+          const int r = u >> 6, i = u & 63;
+          const int64_t qi = qrow(r) * kD;
+          float x0 = load_elem(a.q, a.q_dtype, qi + i), x1 = load_elem(a.q, a.q_dtype, qi + i + kD / 2);
+          if (rope) {
+            const int pos = a.q_pos[bb];
+            if (pos < 0 && a.d_status) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
+            double sn, cs;
+            sincos(dev::rope_angle(pos, i, kD, a.rope_base), &sn, &cs);
+            const double r0 = double(x0) * cs - double(x1) * sn, r1 = double(x0) * sn + double(x1) * cs;
+            x0 = static_cast<float>(r0);
+            x1 = static_cast<float>(r1);
+          }
+          qx[r * kD + i] = x0;
+          qx[r * kD + i + kD / 2] = x1;
         }
-        float vm = 0.f;
-        for (int64_t t = tb + lrow; t < te; t += kTT) vm = fmaxf(vm, __ldg(a.vnorm + row0 + t));
-        loc[12] = vm;
+        named_sync(2, 384);
+        const int i = u & 127, rr = 2 * ((u >> 7) & 1);
+        // q_rot = Pi_K qx, then s = S q_rot.
+        matvec4_split(a.PiK + int64_t(kv) * a.pi_stride, qx, qr, pp, u);
+        matvec4_split(a.S, qr, sv, pp, u);
+        // Row scales: warp w8 = u / 32 covers row w8 / 2, coordinates of half w8 % 2.
+        if (work) {
+          const int w8 = u >> 5, r = w8 >> 1, i0 = (w8 & 1) * 64 + lane;
+          float mq = 0.f, ms = 0.f, ssm = 0.f;
 #pragma unroll
-        for (int u = 0; u < 13; ++u) {
-          const float x = (u >= 8 && u < 12) ? warp_sum(loc[u]) : warp_max(loc[u]);
-          if (lane == 0) gred[cw * 16 + u] = x;
+          for (int k = 0; k < 2; ++k) {
+            const int ii = i0 + 32 * k;
+            const float jsc = __uint_as_float(static_cast<uint32_t>(127 - (ii & 7)) << 23);   // 2^-(i mod 8)
+            mq = fmaxf(mq, fabsf(qr[r * kD + ii]));
+            ms = fmaxf(ms, fabsf(sv[r * kD + ii]) * jsc);
+            ssm += sv[r * kD + ii];
+          }
+          mq = warp_max(mq);
+          ms = warp_max(ms);
+          ssm = warp_sum(ssm);
+          if (lane == 0) {
+            red[w8 * 16 + 0] = mq;
+            red[w8 * 16 + 1] = ms;
+            red[w8 * 16 + 2] = ssm;
+          }
         }
-        wg_sync(bar_id);
-        float tot[13];
+        named_sync(2, 384);
+        if (work) {
+          float sq[2], ss[2];
 #pragma unroll
-        for (int u = 0; u < 13; ++u) {
-          float x = gred[u];
-#pragma unroll
-          for (int w2 = 1; w2 < 4; ++w2) x = (u >= 8 && u < 12) ? x + gred[w2 * 16 + u] : fmaxf(x, gred[w2 * 16 + u]);
-          tot[u] = x;
-        }
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          sq[r] = tot[r] > 0.f ? tot[r] / 127.f : 1.f;
-          ss[r] = tot[4 + r] > 0.f ? tot[4 + r] / 127.f : 1.f;
-          ssum[r] = tot[8 + r];
-        }
-        // Weights p ||v|| <= max ||v|| of the item (p <= 1): three int8 limbs.
-        sp = tot[12] > 0.f ? tot[12] / 127.f : 1.f;
-        if (wg == 0) {
+          for (int k = 0; k < 2; ++k) {
+            const int r = rr + k;
+            const float mq = fmaxf(red[(2 * r) * 16 + 0], red[(2 * r + 1) * 16 + 0]);
+            const float ms = fmaxf(red[(2 * r) * 16 + 1], red[(2 * r + 1) * 16 + 1]);
+            sq[k] = mq > 0.f ? mq / 127.f : 1.f;
+            ss[k] = ms > 0.f ? ms / 127.f : 1.f;
+          }
+          if (u < kRows) {
+            const int r = u;
+            const float mq = fmaxf(red[(2 * r) * 16 + 0], red[(2 * r + 1) * 16 + 0]);
+            const float ms = fmaxf(red[(2 * r) * 16 + 1], red[(2 * r + 1) * 16 + 1]);
+            const float sqr = mq > 0.f ? mq / 127.f : 1.f, ssr = ms > 0.f ? ms / 127.f : 1.f;
+            segk[r] = a.scale * k_scale * sqr;                                   // mse scale
+            segk[4 + r] = 2.f * ssr;                                             // sign-sum scale
+            segk[8 + r] = red[(2 * r) * 16 + 2] + red[(2 * r + 1) * 16 + 2];     // sum s
+          }
           // B tiles: B1/B2/B3 rows 4 r + w hold limb w, w-1, w-2 of q_rot row r;
           // Bs rows 4 r + l hold limb l of s' at K position 16 (i mod 8) + i / 8.
           unsigned char* bt = sm + Sm::kOffB + ib * 4 * 2048;
-          const int ks = 16 * (crd & 7) + (crd >> 3);
+          const int ks = 16 * (i & 7) + (i >> 3);
+          const float jsc = __uint_as_float(static_cast<uint32_t>(127 - (i & 7)) << 23);
 #pragma unroll
-          for (int r = 0; r < kRowsTc; ++r) {
+          for (int k = 0; k < 2; ++k) {
+            const int r = rr + k;
             int lq[4], ls[4];
-            limbs4(qv[r] / sq[r], lq);
-            limbs4(sv[r] * jscale / ss[r], ls);
+            limbs4(qr[r * kD + i] / sq[k], lq);
+            limbs4(sv[r * kD + i] * jsc / ss[k], ls);
 #pragma unroll
             for (int w2 = 0; w2 < 4; ++w2) {
-              bt[sw_byte(4 * r + w2, crd)] = static_cast<unsigned char>(static_cast<int8_t>(lq[w2]));
-              bt[2048 + sw_byte(4 * r + w2, crd)] =
-                  static_cast<unsigned char>(static_cast<int8_t>(w2 >= 1 ? lq[w2 - 1] : 0));
-              bt[4096 + sw_byte(4 * r + w2, crd)] =
-                  static_cast<unsigned char>(static_cast<int8_t>(w2 >= 2 ? lq[w2 - 2] : 0));
+              bt[sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(lq[w2]));
+              bt[2048 + sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(w2 >= 1 ? lq[w2 - 1] : 0));
+              bt[4096 + sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(w2 >= 2 ? lq[w2 - 2] : 0));
               bt[6144 + sw_byte(4 * r + w2, ks)] = static_cast<unsigned char>(static_cast<int8_t>(ls[w2]));
             }
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&b_full[ib]);
+          if (lane == 0) mbar_arrive(&bt_full[ib]);
         }
+        named_sync(2, 384);     // segk visible to all groups; qx/qr/sv free again
       }
-      const float inv_sp = 1.f / sp;
-      float kq[kRowsTc], ks2[kRowsTc];
-      const float kr = a.scale * alpha;
+      if (is_val) {
+        // ------------------------------------------------ value warps
+        const int crd = lrow;                     // coordinate (fold, combine)
+        float acc[2][kRows], m_acc[2][kRows];
 #pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) {
-        kq[r] = a.scale * k_scale * sq[r];
-        ks2[r] = 2.f * ss[r];
-      }
-      // Running maximum and sum of the item's even and odd tiles, kept apart:
-      // the value warps accumulate the two parities separately and each
-      // leaves its own partial record.
-      // m_run / l_part: state of the parity of the tile being processed;
-      // m_oth / l_oth: the other parity's (swapped after every tile).
-      float m_run[kRowsTc], l_part[kRowsTc], m_oth[kRowsTc], l_oth[kRowsTc];
+        for (int g = 0; g < 2; ++g)
 #pragma unroll
-      for (int r = 0; r < kRowsTc; ++r) {
-        m_run[r] = m_oth[r] = -INFINITY;
-        l_part[r] = l_oth[r] = 0.f;
-      }
-      const int j0 = j;
-      // Norms are loaded one tile ahead.
-      float kn_n = 0.f, rn_n = 0.f, vn_n = 0.f;
-      if (lrow < te - tb) {
-        kn_n = __ldg(a.knorm + row0 + tb + lrow);
-        rn_n = __ldg(a.krnorm + row0 + tb + lrow);
-        vn_n = __ldg(a.vnorm + row0 + tb + lrow);
-      }
-      for (int tj = 0; tj < nt_tiles; ++tj) {
-        const int jt = j0 + tj;
-        const int b = jt & 1;
-        const int64_t t0 = tb + int64_t(tj) * kTT;
-        const int nt = static_cast<int>((te - t0 < kTT) ? te - t0 : kTT);
-        const bool valid = lrow < nt;
-        const float kn = kn_n, rn = rn_n, vn = vn_n;
-        if (t0 + kTT + lrow < te) {
-          kn_n = __ldg(a.knorm + row0 + t0 + kTT + lrow);
-          rn_n = __ldg(a.krnorm + row0 + t0 + kTT + lrow);
-          vn_n = __ldg(a.vnorm + row0 + t0 + kTT + lrow);
-        }
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (jt >> 1) & 1));
-        tc_fence_after();
-        uint32_t d[32];
-        tmem_ld32(lane_addr + kColDs + b * 32, d);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ds_free[b]);
-        float score[kRowsTc];
-        bool need = false;
+          for (int r = 0; r < kRows; ++r) {
+            acc[g][r] = 0.f;
+            m_acc[g][r] = -INFINITY;
+          }
+        // Folds group g's current TMEM region (closed; running maxima m_seg in
+        // effect for its tiles) into the registers, then moves to the other.
+        auto fold = [&](int g, const float (&m_seg)[kRows]) -> bool {
+          const int X = 2 * g + vcur[g];
+          if (!__all_sync(0xffffffffu, mbar_wait(&reg_done[X], closes[X] & 1))) return false;
+          tc_fence_after();
+          uint32_t dv[32];
+          tmem_ld32(lane_addr + kColDo + X * 32, dv);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&reg_free[X]);
+          ++closes[X];
+          vcur[g] ^= 1;
 #pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          // weights 0, 1, 2 of the key limb products (weight 3 is below 1e-6)
-          const float mse = limb_sum3(d + 4 * r);
-          const float sgn = limb_sum4(d + 16 + 4 * r);
-          const float qjl = fmaf(ks2[r], sgn, -ssum[r]);
-          score[r] = valid ? fmaf(kq[r] * kn, mse, kr * rn * qjl) : -INFINITY;
-          need |= score[r] > m_run[r];
-        }
-        if (a.scores_out && valid) {
+          for (int r = 0; r < kRows; ++r) {
+            float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-          for (int r = 0; r < kRowsTc; ++r) a.scores_out[qrow[r] * sh.n_ctx + t0 + lrow] = score[r];
-        }
-        float corr[kRowsTc];
+            for (int w8 = 3; w8 >= 0; --w8) {
+              v0 = fmaf(v0, 256.f, static_cast<float>(static_cast<int32_t>(dv[4 * r + w8])));
+              v1 = fmaf(v1, 256.f, static_cast<float>(static_cast<int32_t>(dv[16 + 4 * r + w8])));
+            }
+            const float val = v_scale * fmaf(v1, 1.f / 128.f, v0) * (1.f / 16777216.f);
+            const float c = (m_acc[g][r] == -INFINITY) ? 0.f : ex2(m_acc[g][r] - m_seg[r]);
+            acc[g][r] = fmaf(acc[g][r], c, val);
+            m_acc[g][r] = m_seg[r];
+          }
+          return true;
+        };
+        // Waits for the record of tile jj (CTA-local index).
+        auto rec_ready = [&](int jj) -> bool {
+          volatile uint32_t* rc = recs + (jj & 7) * 16;
+          bool ok = rc[0] == static_cast<uint32_t>(jj);
+          if (!ok) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!(ok = (rc[0] == static_cast<uint32_t>(jj))) && globaltimer_ns() - t0 < 2000000000ull) {
+            }
+          }
+          const bool all = __all_sync(0xffffffffu, ok);
+          __threadfence_block();
+          return all;
+        };
+        // Reads the softmax's record of tile jj; folds the region it closed.
+        auto take_rec = [&](int jj) -> bool {
+          if (!rec_ready(jj)) return false;
+          volatile uint32_t* rc = recs + (jj & 7) * 16;
+          if (rc[1] != 0u) {
+            float mo[kRows];
 #pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) corr[r] = 1.f;
-        // The running maximum moves only when some score of the tile exceeds it.
-        if (wg_sync_or(bar_id, need || !ok || *abort_s != 0)) {
-          if (wg_sync_or(bar_id, !ok || *abort_s != 0)) {
-            if (!ok && lane == 0 && cw == 0) fail();
+            for (int r = 0; r < kRows; ++r) mo[r] = __uint_as_float(rc[2 + r]);
+            if (!fold((jj - j0) & 1, mo)) return false;
+          }
+          return true;
+        };
+        for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
+          const int s = j % kStages;
+          const int b = j & 1;
+          const int row = lrow;                   // token within the tile (operands)
+          if (!__all_sync(0xffffffffu, mbar_wait(&st_full[s], (j / kStages) & 1))) {
+            if (lane == 0) fail();
             stop = true;
             break;
           }
-#pragma unroll
-          for (int r = 0; r < kRowsTc; ++r) {
-            const float mx = warp_max(score[r]);
-            if (lane == 0) gred[cw * 16 + r] = mx;
+          const unsigned char* st = sm + s * Sm::kStageStride;
+          const uint32_t* wrow = reinterpret_cast<const uint32_t*>(st + Sm::kOffVi + row * 48);
+          if (!__all_sync(0xffffffffu, mbar_wait(&vh_free[b], ((j >> 1) & 1) ^ 1))) {
+            if (lane == 0) fail();
+            stop = true;
+            break;
           }
-          wg_sync(bar_id);
+          unsigned char* vh = sm + Sm::kOffVh + b * Sm::kVhBytes;
+          // Row `row` (token) of each limb tile: 128 coordinate bytes, M-major,
+          // 8-token atoms of 1024 bytes. 32 coordinates (12 code bytes, w[0..2])
+          // per iteration; the words shift down after each one.
+          const int atom = row >> 3, r8 = row & 7;
+#pragma unroll 1
+          for (int c2 = 0; c2 < 4; ++c2) {
+            const uint32_t x4[4] = {wrow[3 * c2], wrow[3 * c2 + 1], wrow[3 * c2 + 2], 0u};
 #pragma unroll
-          for (int r = 0; r < kRowsTc; ++r) {
-            float mx = gred[r];
+            for (int cc = 0; cc < 2; ++cc) {          // 16 coordinates = 6 bytes of codes
+              uint32_t o1[4], o2[4];
 #pragma unroll
-            for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, gred[w2 * 16 + r]);
-            const float m_new = fmaxf(m_run[r], mx);
-            corr[r] = (m_run[r] == -INFINITY) ? 0.f : ex2((m_run[r] - m_new) * kLog2e);
-            l_part[r] *= corr[r];
-            m_run[r] = m_new;
+              for (int h = 0; h < 2; ++h) {           // 8 codes per half
+                const int g = 2 * cc + h;
+                const int off = 3 * g, wi = off >> 2, shf = 8 * (off & 3);
+                const uint32_t x = shf == 0 ? x4[wi] : __funnelshift_r(x4[wi], x4[wi + 1], shf);
+                const uint32_t nb = nibbles3(x);
+                o1[2 * h] = prmt(v1t[0], v1t[1], nb);
+                o1[2 * h + 1] = prmt(v1t[0], v1t[1], nb >> 16);
+                o2[2 * h] = prmt(v2t[0], v2t[1], nb);
+                o2[2 * h + 1] = prmt(v2t[0], v2t[1], nb >> 16);
+              }
+              const int c16 = 2 * c2 + cc;
+              const uint32_t off = atom * 1024 + r8 * 128 + ((c16 ^ r8) << 4);
+              *reinterpret_cast<uint4*>(vh + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+              *reinterpret_cast<uint4*>(vh + kTT * 128 + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&st_empty[s]);
+            mbar_arrive(&vh_full[b]);
+          }
+          // The softmax of tile j - 2 is done (its PV product freed this buffer).
+          if (tj >= 2 && !take_rec(j - 2)) {
+            if (lane == 0) fail();
+            stop = true;
+            break;
           }
         }
-        float p[kRowsTc];
+        // Segment end: the last tiles' records, then each group's final region.
+        bool okr = !stop;
+        for (int jj = max(j0, j - 2); jj < j && okr; ++jj) okr = take_rec(jj);
+        bool ran[2] = {false, false};
 #pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          p[r] = valid ? ex2((score[r] - m_run[r]) * kLog2e) : 0.f;
-          l_part[r] += p[r];
-        }
-        // Weight limbs into the P tile (row 3 r + limb, column = token); the
-        // tile's corrections and scale go to ring[jt % 4] for the value warps.
-        if (!__all_sync(0xffffffffu, mbar_wait(&p_free[b], ((jt >> 1) & 1) ^ 1)) && lane == 0) fail();
-        if (lrow == 0) {
-          float* slot = ring + (jt & 3) * 8;
-          reinterpret_cast<float4*>(slot)[0] = make_float4(corr[0], corr[1], corr[2], corr[3]);
-          slot[4] = sp;
-          __threadfence_block();
-          *reinterpret_cast<volatile int*>(slot + 5) = jt;
-        }
-        unsigned char* pt = sm + Sm::kOffP + b * 2048;
-        const float wv = vn * inv_sp;
+        for (int g = 0; g < 2; ++g) {
+          if (!okr || nt_tiles <= g) continue;
+          const int last = j0 + nt_tiles - 1 - ((nt_tiles - 1 - g) & 1);   // the group's last tile
+          float mf[kRows];
+          {
+            volatile uint32_t* rc = recs + (last & 7) * 16;
 #pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          // X = rint(x 2^14) < 2^21 in the low mantissa bits; its base-128
-          // digits are the limbs: x ~ d1 + d2/128 + d3/128^2.
-          const float x = fminf(p[r] * wv, 127.f);
-          const uint32_t X = __float_as_uint(fmaf(x, 16384.f, kMagic)) - 0x4B400000u;
-          pt[poff[3 * r]] = static_cast<unsigned char>(X >> 14);
-          pt[poff[3 * r + 1]] = static_cast<unsigned char>((X >> 7) & 127u);
-          pt[poff[3 * r + 2]] = static_cast<unsigned char>(X & 127u);
+            for (int r = 0; r < kRows; ++r) mf[r] = __uint_as_float(rc[6 + r]);
+          }
+          if (!fold(g, mf)) okr = false;
+          ran[g] = true;     // acc[g] is now relative to the group's final maxima
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[b]);
+        if (!okr) {
+          if (lane == 0) fail();
+          stop = true;
+        }
+        // Partial record: both groups' sums on the larger of their maxima.
 #pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          const float tm = m_run[r], tl = l_part[r];
-          m_run[r] = m_oth[r];
-          l_part[r] = l_oth[r];
-          m_oth[r] = tm;
-          l_oth[r] = tl;
+        for (int r = 0; r < kRows; ++r) {
+          float o = 0.f;
+          const float M = ran[1] ? fmaxf(m_acc[0][r], m_acc[1][r]) : m_acc[0][r];
+          if (ran[0]) o = acc[0][r] * segk[16] * ex2(m_acc[0][r] - M);
+          if (ran[1]) o = fmaf(acc[1][r] * segk[17], ex2(m_acc[1][r] - M), o);
+          a.part[(rec_idx * kRows + r) * kRecFloats + crd] = o;
+        }
+      } else {
+        // ---------------------------------------------- softmax group sgrp
+        float kq[kRows], ks2[kRows], ssum[kRows];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          kq[r] = segk[r];
+          ks2[r] = segk[4 + r];
+          ssum[r] = segk[8 + r];
+        }
+        const float kr = a.scale * alpha;
+        float m_run[kRows], l_part[kRows];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          m_run[r] = -INFINITY;
+          l_part[r] = 0.f;
+        }
+        float inv_v0 = 0.f;
+        for (int k = 0; 2 * k + sgrp < nt_tiles; ++k) {
+          const int tj = 2 * k + sgrp;
+          const int jt = j0 + tj;
+          const int b = jt & 1;
+          const int64_t t0 = (sg.t0 + tj) * kTT;
+          const int nt = static_cast<int>((sh.n_ctx - t0 < kTT ? sh.n_ctx - t0 : int64_t(kTT)));
+          const bool valid = lrow < nt;
+          norm_fetch(k + 3);
+          cp_async_wait<3>();
+          const float* slot = nring + (k & 3) * (3 * kTT);
+          const float kn = slot[lrow], rn = slot[kTT + lrow], vn = slot[2 * kTT + lrow];
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (jt >> 1) & 1));
+          tc_fence_after();
+          // MSE part: weights 1, 1/128, 1/128^2 of the key-limb products
+          // (weight 3 is below 1e-6 of the first); sign part: four limbs.
+          // The two halves are read one after the other (fewer live registers).
+          float mse[kRows], sgn[kRows];
+          {
+            uint32_t d[16];
+            tmem_ld16(lane_addr + kColDs + b * 32, d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              const int32_t m01 = static_cast<int32_t>(d[4 * r]) * 128 + static_cast<int32_t>(d[4 * r + 1]);
+              mse[r] = fmaf(static_cast<float>(static_cast<int32_t>(d[4 * r + 2])), 1.f / 16384.f,
+                            static_cast<float>(m01) * (1.f / 128.f));
+            }
+            tmem_ld16(lane_addr + kColDs + b * 32 + 16, d);
+            tmem_ld_wait();
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              const int32_t e01 = static_cast<int32_t>(d[4 * r]) * 128 + static_cast<int32_t>(d[4 * r + 1]);
+              const int32_t e23 = static_cast<int32_t>(d[4 * r + 2]) * 128 + static_cast<int32_t>(d[4 * r + 3]);
+              sgn[r] = fmaf(static_cast<float>(e23), 1.f / 2097152.f, static_cast<float>(e01) * (1.f / 128.f));
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ds_free[b]);
+          float s2[kRows];
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            const float qjl = fmaf(ks2[r], sgn[r], -ssum[r]);
+            const float mse_r = mse[r];
+            const float sn = fmaf(kq[r] * kn, mse_r, kr * rn * qjl);
+            if (a.scores_out && valid) a.scores_out[qrow(r) * sh.n_ctx + t0 + lrow] = sn;
+            s2[r] = valid ? sn * kLog2e : -INFINITY;
+          }
+          bool flip = false;
+          float m_old[kRows];
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) m_old[r] = m_run[r];
+          float x[kRows], p[kRows];
+          if (k == 0) {
+            // The group's first tile sets its running maxima and V0.
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              const float mx = warp_max(s2[r]);
+              if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + r] = mx;
+            }
+            {
+              const float vm = warp_max(valid ? vn : 0.f);
+              if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + 4] = vm;
+            }
+            named_sync(sbar, 128);
+            float v0 = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < 4; ++w2) v0 = fmaxf(v0, red[(8 + 4 * sgrp + w2) * 16 + 4]);
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              float mx = red[(8 + 4 * sgrp) * 16 + r];
+#pragma unroll
+              for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, red[(8 + 4 * sgrp + w2) * 16 + r]);
+              m_run[r] = mx;
+              m_old[r] = mx;
+            }
+            inv_v0 = v0 > 0.f ? 1.f / v0 : 0.f;
+            if (lrow == 0) segk[16 + sgrp] = v0;
+            named_sync(sbar, 128);
+          }
+          const float wv = vn * inv_v0;
+          bool need = false;
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            p[r] = valid ? ex2(fminf(s2[r] - m_run[r], 100.f)) : 0.f;
+            x[r] = p[r] * wv;
+            need |= !(x[r] <= 64.f) && valid;
+          }
+          // One vote per tile (uniform over the group's four warps): a weight
+          // out of range, or a failed wait / abort anywhere in the group.
+          const bool bad = !ok || *abort_s != 0;
+          if (wg_sync_or(sbar, need || bad)) {
+            if (wg_sync_or(sbar, bad)) {
+              if (!ok && lane == 0) fail();
+              stop = true;
+              break;
+            }
+            // A weight would leave the fixed-point range: move the running
+            // maximum by the whole number of octaves that brings every weight
+            // of the tile back to <= 1.
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              const float z = valid ? (s2[r] - m_run[r]) + __log2f(fmaxf(wv, 1e-30f)) : -INFINITY;
+              const float zm = warp_max(z);
+              if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + r] = zm;
+            }
+            named_sync(sbar, 128);
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              float zm = red[(8 + 4 * sgrp) * 16 + r];
+#pragma unroll
+              for (int w2 = 1; w2 < 4; ++w2) zm = fmaxf(zm, red[(8 + 4 * sgrp + w2) * 16 + r]);
+              const float dl = zm > 0.f ? ceilf(zm) : 0.f;
+              m_run[r] += dl;
+              l_part[r] *= ex2(-dl);
+              p[r] = valid ? ex2(s2[r] - m_run[r]) : 0.f;
+              x[r] = p[r] * wv;
+            }
+            named_sync(sbar, 128);
+            flip = true;
+          }
+          uint32_t X[kRows];
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            l_part[r] += p[r];
+            X[r] = valid ? __float2uint_rn(x[r] * 16777216.f) : 0u;
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(&p_free[b], ((jt >> 1) & 1) ^ 1)) && lane == 0) fail();
+          *reinterpret_cast<uint4*>(sm + Sm::kOffP + b * 2048 + lrow * 16) = make_uint4(X[0], X[1], X[2], X[3]);
+          if (lrow == 0) {
+            volatile uint32_t* rc = recs + (jt & 7) * 16;
+            rc[1] = flip ? 1u : 0u;
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              rc[2 + r] = __float_as_uint(m_old[r]);
+              rc[6 + r] = __float_as_uint(m_run[r]);
+            }
+            __threadfence_block();
+            rc[0] = static_cast<uint32_t>(jt);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[b]);
+        }
+        cp_async_wait<0>();
+        j = j0 + nt_tiles;
+        // Segment end: the group's l per row; its m and l for the record (the
+        // four warps stopped together or not at all).
+        if (!stop) {
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            const float x = warp_sum(l_part[r]);
+            if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + 8 + r] = x;
+          }
+          named_sync(sbar, 128);
+          if (lrow < kRows) {
+            const int r = lrow;
+            const float* rg = red + (8 + 4 * sgrp) * 16 + 8 + r;
+            segk[20 + 8 * sgrp + r] = m_run[r];
+            segk[24 + 8 * sgrp + r] = rg[0] + rg[16] + rg[32] + rg[48];
+          }
         }
       }
-      j = j0 + nt_tiles;
-      if (stop) break;
-      // Softmax statistics of the two partials (the value warps write acc).
-      // m_run / l_part now hold the parity of tile j0 + nt_tiles, m_oth / l_oth
-      // the other one.
-      const int par_run = (j0 + nt_tiles) & 1;
+      // ---------------- arrival; the stream's last segment merges. All groups
+      // pass the same barriers whether or not they stopped; the decision to
+      // quit is taken once, after the first of them.
+      __threadfence();
+      named_sync(2, 384);
+      if (u == 0) {
+        merge_s[1] = *abort_s != 0 ? 1 : 0;
+        // m and l of the segment's record from the two groups' (a group
+        // without tiles has m = -inf, l = 0).
 #pragma unroll
-      for (int par = 0; par < 2; ++par) {
-        const bool use_run = par == par_run;
-        float lsum[kRowsTc];
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) {
-          const float x = warp_sum(use_run ? l_part[r] : l_oth[r]);
-          if (lane == 0) gred2[cw * 4 + r] = x;
+        for (int r = 0; r < kRows; ++r) {
+          const float m0 = segk[20 + r], l0 = segk[24 + r];
+          const float m1 = nt_tiles > 1 ? segk[28 + r] : -INFINITY, l1 = nt_tiles > 1 ? segk[32 + r] : 0.f;
+          const float M = fmaxf(m0, m1);
+          float* pr = a.part + (rec_idx * kRows + r) * kRecFloats;
+          pr[kD] = M;
+          pr[kD + 1] = l0 * ex2(m0 - M) + (nt_tiles > 1 ? l1 * ex2(m1 - M) : 0.f);
         }
-        wg_sync(bar_id);
-#pragma unroll
-        for (int r = 0; r < kRowsTc; ++r) lsum[r] = gred2[r] + gred2[4 + r] + gred2[8 + r] + gred2[12 + r];
-        wg_sync(bar_id);
-        if (lrow == 0) {
-          // record 2 split + parity of the tiles' index j
-          const int rec = 2 * split + par;
-#pragma unroll
-          for (int r = 0; r < kRowsTc; ++r) {
-            float* pr = a.part + (qrow[r] * sh.n_parts + rec) * (kD + 2);
-            pr[kD] = use_run ? m_run[r] : m_oth[r];
-            pr[kD + 1] = lsum[r];
-          }
+        __threadfence();
+        const int64_t vf = vof(part, sg.s * part.Ts), vl = vof(part, (sg.s + 1) * part.Ts - 1);
+        const int nseg = static_cast<int>(vl - vf + 1);
+        const int old = atomicAdd(A.counters + sg.s, 1);
+        const int last = old == nseg - 1;
+        if (last) __threadfence();
+        merge_s[0] = last ? 1 : 0;
+        if (last) {
+          reinterpret_cast<int64_t*>(red)[0] = vf;
+          reinterpret_cast<int64_t*>(red)[1] = vl;
         }
       }
+      named_sync(2, 384);
+      if (merge_s[1]) break;
+      if (merge_s[0]) {
+        // All three groups: rows merged by the value group (thread =
+        // coordinate), then out = Pi_V^T o_rot with the input coordinates j
+        // split in three (thread = output coordinate), partial sums in smem.
+        const int64_t vf = reinterpret_cast<const int64_t*>(red)[0], vl = reinterpret_cast<const int64_t*>(red)[1];
+        const int crd = u & 127, part3 = u >> 7;
+        if (is_val) {
+          // The stream's records, four at a time with all loads in flight,
+          // merged online (running maximum, sum and rotated output per row).
+          float M[kRows], L[kRows], O[kRows];
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            M[r] = -INFINITY;
+            L[r] = 0.f;
+            O[r] = 0.f;
+          }
+          for (int64_t v0 = vf; v0 <= vl; v0 += 4) {
+            float mk[4][kRows], lk[4][kRows], ok[4][kRows];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+              for (int r = 0; r < kRows; ++r) {
+                const bool has = v0 + kk <= vl;
+                const float* pr = a.part + ((v0 + kk + sg.s) * kRows + r) * kRecFloats;
+                mk[kk][r] = has ? __ldcg(pr + kD) : -INFINITY;
+                lk[kk][r] = has ? __ldcg(pr + kD + 1) : 0.f;
+                ok[kk][r] = has ? __ldcg(pr + crd) : 0.f;
+              }
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) {
+              float Mn = M[r];
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) Mn = fmaxf(Mn, mk[kk][r]);
+              const float c = M[r] == -INFINITY ? 0.f : ex2(M[r] - Mn);
+              L[r] *= c;
+              O[r] *= c;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const float wgt = mk[kk][r] == -INFINITY ? 0.f : ex2(mk[kk][r] - Mn);
+                L[r] = fmaf(lk[kk][r], wgt, L[r]);
+                O[r] = fmaf(ok[kk][r], wgt, O[r]);
+              }
+              M[r] = Mn;
+            }
+          }
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) qx[r * kD + crd] = L[r] > 0.f ? O[r] / L[r] : 0.f;
+        }
+        named_sync(2, 384);
+        const float* PV = a.PiV + int64_t(kv) * a.pi_stride;
+        const int j_lo = part3 * 43, j_n = part3 == 2 ? 42 : 43;
+        float o4[kRows] = {0.f, 0.f, 0.f, 0.f};
+        {
+          float pv[43];
+#pragma unroll
+          for (int k = 0; k < 43; ++k) pv[k] = k < j_n ? __ldg(PV + int64_t(j_lo + k) * kD + crd) : 0.f;
+#pragma unroll
+          for (int k = 0; k < 43; ++k) {
+            const int jj = j_lo + (k < j_n ? k : 0);
+#pragma unroll
+            for (int r = 0; r < kRows; ++r) o4[r] = fmaf(pv[k], qx[r * kD + jj], o4[r]);
+          }
+        }
+        // Parts 1 and 2 leave their sums in qr / sv; part 0 (the value group)
+        // adds them and stores the rows.
+        if (part3 > 0) {
+          float* dst = part3 == 1 ? qr : sv;
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) dst[r * kD + crd] = o4[r];
+        }
+        named_sync(2, 384);
+        if (part3 == 0) {
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            const float v = o4[r] + qr[r * kD + crd] + sv[r * kD + crd];
+            const int64_t oi = qrow(r) * kD + crd;
+            if (a.out_dtype == 0) reinterpret_cast<float*>(a.out)[oi] = v;
+            else reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(v);
+          }
+          if (crd == 0) A.counters[sg.s] = 0;    // ready for the next call
+        }
+      }
+      named_sync(2, 384);                         // qx is the next prologue's again
     }
   }
 
@@ -901,45 +1245,86 @@ __global__ void __launch_bounds__(kThreadsTc, 1) decode_tc_kernel(TcDecodeArgs A
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWScore) {
     tc_fence_after();
     __syncwarp();
-    tmem_dealloc(tmem, kTmemColsTc);
+    tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+struct FusedPlan {
+  int64_t T, Ts, streams;
+  int V;
+  size_t off_part, bytes;
+};
+// Partition and workspace of a call on `grid` CTAs: [arrival counters, one per
+// stream | partial records, one per (virtual CTA, stream) pair index v + s].
+FusedPlan fused_plan(const DecodeShape& s, int grid) {
+  FusedPlan p{};
+  p.streams = int64_t(s.batch) * s.hkv;
+  p.Ts = (s.n_ctx + kTT - 1) / kTT;
+  p.T = p.streams * p.Ts;
+  const int64_t vmin = (p.T + kMaxSegTiles - 1) / kMaxSegTiles;
+  // Every physical CTA gets the same number of virtual ones.
+  p.V = static_cast<int>(((std::max<int64_t>(vmin, 1) + grid - 1) / grid) * grid);
+  p.off_part = ((size_t(p.streams) * sizeof(int) + 255) / 256) * 256;
+  p.bytes = p.off_part + size_t(p.V + p.streams) * kRows * kRecFloats * sizeof(float);
+  return p;
+}
+
+int fused_grid(const DecodeShape& s, int sms) {
+  const int64_t T = int64_t(s.batch) * s.hkv * ((s.n_ctx + kTT - 1) / kTT);
+  return static_cast<int>(std::min<int64_t>(std::min(sms, kMaxGrid), T));
 }
 
 }  // namespace
 
 bool tc_decode_supported(const DecodeArgs& v) {
   const DecodeShape& s = v.sh;
-  if (s.d != kD || s.vbits != 3 || s.rows_per_cta != kRowsTc || s.row_blocks != 1) return false;
+  if (s.d != kD || s.vbits != 3 || s.nq != 1 || s.hq != kRows * s.hkv) return false;
   if (s.kbits < 2 || s.kbits > 4) return false;
-  // Bulk copies need 16-byte aligned sources: plane bases and stream offsets.
+  // Bulk copies need 16-byte aligned sources: plane bases and stream offsets
+  // (rows are multiples of 16 bytes); the prologue reads Pi_K and S rows as
+  // float4.
   if (!aligned(v.kidx, 16) || !aligned(v.ksign, 16) || !aligned(v.vidx, 16)) return false;
+  if (!aligned(v.PiK, 16) || !aligned(v.S, 16) || v.pi_stride % 4 != 0) return false;
   return true;
 }
 
-cudaError_t tc_decode_launch(const DecodeArgs& v, cudaStream_t st) {
-  TcDecodeArgs A{};
-  A.v = v;
-  A.n_items = static_cast<int>(int64_t(v.sh.batch) * v.sh.hkv * v.sh.n_splits);
+size_t tc_decode_workspace_bytes(const DecodeShape& s) {
+  if (s.d != kD || s.vbits != 3 || s.nq != 1 || s.hq != kRows * s.hkv) return 0;
+  return fused_plan(s, fused_grid(s, kMaxGrid)).bytes;     // covers every grid <= kMaxGrid
+}
+
+cudaError_t tc_decode_launch(const DecodeArgs& v, void* workspace, cudaStream_t st) {
   int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = A.n_items < sms ? A.n_items : sms;
-  cudaError_t e;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int grid = fused_grid(v.sh, sms);
+  const FusedPlan p = fused_plan(v.sh, grid);
+  FusedArgs A{};
+  A.v = v;
+  A.T = p.T;
+  A.Ts = p.Ts;
+  A.V = p.V;
+  A.counters = static_cast<int*>(workspace);
+  A.v.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.off_part);
+  e = cudaMemsetAsync(A.counters, 0, size_t(p.streams) * sizeof(int), st);
+  if (e != cudaSuccess) return e;
   switch (v.sh.kbits) {
     case 2:
-      e = cudaFuncSetAttribute(decode_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSm<2>::kBytes);
-      if (e == cudaSuccess) decode_tc_kernel<2><<<grid, kThreadsTc, TcSm<2>::kBytes, st>>>(A);
+      e = cudaFuncSetAttribute(decode_fused_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, FSm<2>::kBytes);
+      if (e == cudaSuccess) decode_fused_kernel<2><<<grid, kThreads, FSm<2>::kBytes, st>>>(A);
       break;
     case 3:
-      e = cudaFuncSetAttribute(decode_tc_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSm<3>::kBytes);
-      if (e == cudaSuccess) decode_tc_kernel<3><<<grid, kThreadsTc, TcSm<3>::kBytes, st>>>(A);
+      e = cudaFuncSetAttribute(decode_fused_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, FSm<3>::kBytes);
+      if (e == cudaSuccess) decode_fused_kernel<3><<<grid, kThreads, FSm<3>::kBytes, st>>>(A);
       break;
     default:
-      e = cudaFuncSetAttribute(decode_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSm<4>::kBytes);
-      if (e == cudaSuccess) decode_tc_kernel<4><<<grid, kThreadsTc, TcSm<4>::kBytes, st>>>(A);
+      e = cudaFuncSetAttribute(decode_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, FSm<4>::kBytes);
+      if (e == cudaSuccess) decode_fused_kernel<4><<<grid, kThreads, FSm<4>::kBytes, st>>>(A);
       break;
   }
   if (e != cudaSuccess) return e;

@@ -15,7 +15,7 @@ struct DecodeShape {
   int rows_per_cta;   // R
   int row_blocks;     // (hq/hkv*nq) / R
   int n_splits;
-  int n_parts;        // partial records per query row: n_splits, or 2 n_splits (tensor-core path)
+  int n_parts;        // partial records per query row (CUDA-core path): n_splits
   int64_t chunk;      // tokens per split (multiple of kT)
   int64_t n_rows;     // batch*hq*nq
 };
@@ -42,14 +42,18 @@ struct DecodeArgs {
   void* out;
   int out_dtype;
   float* scores_out;
-  float* qs;     // [n_rows][2][d]  q_rot then s
-  float* part;   // [n_rows][n_parts][d + 2]  acc..., m, l
+  float* qs;     // CUDA-core path: [n_rows][2][d]  q_rot then s
+  float* part;   // partial records (layout per path)
   int32_t* d_status;
 };
 
-// Tensor-core decode (tq_decode_tc.cu): d = 128, four query rows per KV
-// stream, 3-bit values, 2-4 bit keys.
+// Fused tensor-core decode (tq_decode_tc.cu): d = 128, a GQA group of four
+// query heads with one query each, 3-bit values, 2-4 bit keys; one launch
+// (after a memset of its arrival counters) computes the whole call.
 bool tc_decode_supported(const DecodeArgs& a);
-cudaError_t tc_decode_launch(const DecodeArgs& a, cudaStream_t st);
+// Workspace bytes of the fused path for this shape (0 if the shape is not one
+// it runs).
+size_t tc_decode_workspace_bytes(const DecodeShape& s);
+cudaError_t tc_decode_launch(const DecodeArgs& a, void* workspace, cudaStream_t st);
 
 }  // namespace tq

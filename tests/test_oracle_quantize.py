@@ -43,6 +43,30 @@ def test_rope_is_a_rotation_with_relative_position_property():
         assert abs(oq.rope(q, m, base) @ oq.rope(k, m + 5, base) - ref) < 1e-11
 
 
+def test_rope_literal_values_of_the_published_definition():
+    # Rotate-half RoPE as published (RoFormer, Su et al., section 3.4.2, with
+    # theta_i = base^(-2(i-1)/d) for 1-based pair index i; the pairing of
+    # channel i with channel i + d/2 is the rotate-half convention). Worked by
+    # hand at d = 4, base = 1e4, position 1: the two pair angles are 1 and
+    # 1e4^(-1/2) = 0.01, so e_0 -> (cos 1, 0, sin 1, 0), e_1 -> (0, cos .01, 0,
+    # sin .01), e_2 -> (-sin 1, 0, cos 1, 0), e_3 -> (0, -sin .01, 0, cos .01).
+    c1, s1 = 0.5403023058681398, 0.8414709848078965          # cos 1, sin 1
+    c2, s2 = 0.9999500004166653, 0.009999833334166664        # cos .01, sin .01
+    expect = np.array([[c1, 0.0, s1, 0.0],
+                       [0.0, c2, 0.0, s2],
+                       [-s1, 0.0, c1, 0.0],
+                       [0.0, -s2, 0.0, c2]])
+    np.testing.assert_allclose(oq.rope(np.eye(4), np.ones(4), 1e4), expect, atol=1e-15)
+    # d = 8, position 3: angles 3, 0.3, 0.03, 0.003 (exponents 0, -1/4, -1/2,
+    # -3/4 of 1e4). A wrong exponent such as -i/d or -2(i+1)/d moves them.
+    ang = np.array([3.0, 0.3, 0.03, 0.003])
+    out = oq.rope(np.eye(8)[:4], np.full(4, 3), 1e4)
+    for i in range(4):
+        want = np.zeros(8)
+        want[i], want[i + 4] = math.cos(ang[i]), math.sin(ang[i])
+        np.testing.assert_allclose(out[i], want, atol=1e-14)
+
+
 def test_rope_then_rotation_preserves_scores():
     # (Pi R_i q)^T (Pi R_j k) = q^T R_i^T R_j k.
     d = 64
