@@ -1,6 +1,7 @@
 // Fused tensor-core decode attention (sm_100a, tcgen05 kind::i8) for d = 128,
 // four query rows per KV stream (a GQA group of four heads, one query each),
-// 3-bit values and 2-4-bit keys: the whole call in one launch.
+// 3-bit values and 2-4-bit keys: the whole call in two launches (a query-side
+// prologue and the main kernel) after a memset of the arrival counters.
 //
 // Sources: gist.science "TurboESM ..." section 2E (one fused kernel unpacks
 // the codes, applies the QJL correction and the inverse rotation and runs an
@@ -12,8 +13,10 @@
 //               512 tiles: cut again). A range splits into segments at stream
 //               ends; each segment leaves one partial record (m, l, acc) per
 //               query row.
-//   Prologue    per segment: q_rot = Pi_K RoPE(q), s = S q_rot and their int8
-//               limbs as the B operands of the score MMAs.
+//   Prologue    a small kernel before the main one: per stream q_rot =
+//               Pi_K RoPE(q), s = S q_rot and their int8 limbs as the B
+//               operands of the score MMAs; the main kernel's loader copies a
+//               segment's share in with one bulk copy.
 //   Scores      A (TMEM, one lane per token): the key codebook value of every
 //               coordinate as three int8 limbs, c = sc (a1 + a2/128 + a3/128^2),
 //               and the sign chunk, masked in place (byte 16 j + b = byte b of
@@ -41,7 +44,6 @@
 //   warps 4-7    key operands into TMEM            (thread = token)
 //   warps 8-11   value operands into smem, folds, combine (thread = token / coordinate)
 //   warps 12-15  scores, softmax, weights          (thread = token)
-// Warps 8-15 also compute the segment prologue together.
 // Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT and the CTA
 // drains its copies and MMAs before it frees TMEM and returns.
 #include <cuda.h>
@@ -66,13 +68,19 @@ using dev::warp_sum;
 constexpr int kD = 128;
 constexpr int kTT = 128;               // tokens per tile
 constexpr int kStages = 4;
+constexpr int kNVh = 3;                // value operand / P buffers (tile j uses j % 3)
+// Per stream, the query side of the score MMAs (written by the prologue
+// kernel): the B tiles B1 | B2 | B3 | Bs (4 x 2 KB, K-major, 128-byte swizzle)
+// and 16 floats: scale*sq[4], 2*ss[4], sum s[4], pad.
+constexpr int kQPrepBytes = 4 * 2048 + 64;
+constexpr int kQPrepStride = 8448;      // bytes between streams in the workspace (256-aligned)
+constexpr int kBStride = 9216;          // bytes between the two smem copies (1024-aligned)
 constexpr int kThreads = 640;          // 20 warps
 constexpr int kRows = 4;               // query rows per stream
 constexpr int kMaxSegTiles = 512;      // PV accumulators: < 2^31 over this many tiles
 constexpr int kMaxGrid = 256;
 constexpr int kRecFloats = 132;        // partial record: acc[128], m, l, pad
-constexpr int kWLoader = 0, kWScore = 1, kWPv = 2, kWKey0 = 4, kWVal0 = 8, kWSoft0 = 12;   // softmax groups: 12-15, 16-19
-constexpr int kSegFloats = 48;         // per-segment constants
+constexpr int kWLoader = 0, kWScore = 1, kWPv = 2, kWKey0 = 4, kWVs0 = 12;   // key groups 4-7, 8-11; value+softmax groups 12-15, 16-19
 
 // TMEM columns (32-bit): A_score x2 at 0, 128 (a1 | a2 | a3 | sgn, 32 each);
 // D_score x2 at 256, 288 (mse 16 | sgn 16); D_o regions x4 at 320 + 32 X
@@ -92,19 +100,18 @@ struct FSm {
   static constexpr int kOffVi = kOffKs + kTT * 16;                 // value index rows
   static constexpr int kStageBytes = kOffVi + kTT * 48;
   static constexpr int kStageStride = ((kStageBytes + 1023) / 1024) * 1024;
-  static constexpr int kOffVh = kStages * kStageStride;            // 2 buffers x 2 limbs x 16 KB
+  static constexpr int kOffVh = kStages * kStageStride;            // kNVh buffers x 2 limbs x 16 KB
   static constexpr int kVhBytes = 2 * kTT * 128;
-  static constexpr int kOffP = kOffVh + 2 * kVhBytes;              // 2 x [128 tokens][16 B]
-  static constexpr int kOffB = kOffP + 2 * 2048;                   // 2 segments x (B1 | B2 | B3 | Bs)
-  static constexpr int kOffQ = kOffB + 2 * 4 * 2048;               // qx, qr, sv: [4][128] floats each
-  static constexpr int kOffPP = kOffQ + 3 * kRows * kD * 4;        // [3][4][128] floats: matvec partials
-  static constexpr int kOffRed = kOffPP + 3 * kRows * kD * 4;      // [16][16] floats
-  static constexpr int kOffSeg = kOffRed + 16 * 16 * 4;            // [2][kSegFloats] per-segment constants
-  static constexpr int kOffNrm = kOffSeg + 2 * kSegFloats * 4;     // [2 groups][4 slots][3][128] norms
+  static constexpr int kOffP = kOffVh + kNVh * kVhBytes;           // kNVh x [128 tokens][16 B]
+  static constexpr int kOffB = kOffP + kNVh * 2048;                // 2 segments x (B1 | B2 | B3 | Bs | consts)
+  static constexpr int kOffQ = kOffB + 2 * kBStride;               // qx, qr, sv: [4][128] floats each (combine)
+  static constexpr int kOffPP = kOffQ + 3 * kRows * kD * 4;        // [4][128] floats: matvec partials
+  static constexpr int kOffRed = kOffPP + kRows * kD * 4;          // [16][16] floats
+  static constexpr int kOffNrm = kOffRed + 16 * 16 * 4;            // [2 groups][4 slots][3][128] norms
   static constexpr int kOffRec = kOffNrm + 2 * 4 * 3 * kTT * 4;    // [8][16] words: tile records
   static constexpr int kOffTab = kOffRec + 8 * 16 * 4;             // limb tables (20 words) + 2 scales
   static constexpr int kOffBar = kOffTab + 32 * 4;
-  static constexpr int kNumBars = 2 * kStages + 7 * 2 + 4 + 4 + 2;
+  static constexpr int kNumBars = 2 * kStages + 5 * 2 + 2 * kNVh + 4 + 4 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64 + 1024;               // + alignment slack
 };
@@ -116,6 +123,7 @@ struct FusedArgs {
   int64_t T, Ts;       // tiles in all, tiles per stream
   int V;               // virtual CTAs
   int* counters;       // [streams] arrivals (zero at launch)
+  unsigned char* qprep;  // [streams][kQPrepStride] query side of the score MMAs
 };
 
 // int8 limbs of the key codebook (three) and the value codebook (two),
@@ -264,34 +272,35 @@ __device__ __forceinline__ uint64_t desc_mn_noswz(uint32_t saddr) {
 }
 
 // y[r][i] = sum_j M[i][j] x[r][j] for four rows (x, y: shared [4][128]) on
-// 384 threads: thread u takes output coordinate i = u % 128 and the input
-// coordinates of part u / 128 (44, 44, 40 of them, whole float4s), with all
-// of its row loads in flight; the three partial sums meet in pp [3][4][128].
-// Two barriers of the 384 threads (id 2).
+// 256 threads: thread u takes output coordinate i = u % 128 and the input
+// coordinates of half u / 128 (64 of them, 16 float4s), with all of its row
+// loads in flight; the two partial sums meet in pp [2][4][128]. Two barriers
+// of the 256 threads (id 2).
 __device__ __forceinline__ void matvec4_split(const float* __restrict__ M, const float* x, float* y, float* pp, int u) {
   const int i = u & 127, part = u >> 7;
-  const int j4_0 = part * 11, n4 = part == 2 ? 10 : 11;
-  const float4* row = reinterpret_cast<const float4*>(M + int64_t(i) * kD) + j4_0;
-  float4 mv[11];
+  const float4* row = reinterpret_cast<const float4*>(M + int64_t(i) * kD) + part * 16;
+  float4 mv[16];
 #pragma unroll
-  for (int k = 0; k < 11; ++k) mv[k] = k < n4 ? __ldg(row + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < 16; ++k) mv[k] = __ldg(row + k);
   float acc[kRows] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int k = 0; k < 11; ++k) {
+  for (int k = 0; k < 16; ++k) {
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
-      const float4 xv = reinterpret_cast<const float4*>(x + r * kD)[j4_0 + (k < n4 ? k : 0)];
+      const float4 xv = reinterpret_cast<const float4*>(x + r * kD)[part * 16 + k];
       acc[r] = fmaf(mv[k].x, xv.x, fmaf(mv[k].y, xv.y, fmaf(mv[k].z, xv.z, fmaf(mv[k].w, xv.w, acc[r]))));
     }
   }
+  if (part == 1) {
 #pragma unroll
-  for (int r = 0; r < kRows; ++r) pp[(part * kRows + r) * kD + i] = acc[r];
-  named_sync(2, 384);
-  if (u < 128) {
-#pragma unroll
-    for (int r = 0; r < kRows; ++r) y[r * kD + i] = pp[r * kD + i] + pp[(kRows + r) * kD + i] + pp[(2 * kRows + r) * kD + i];
+    for (int r = 0; r < kRows; ++r) pp[r * kD + i] = acc[r];
   }
-  named_sync(2, 384);
+  named_sync(2, 256);
+  if (part == 0) {
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) y[r * kD + i] = acc[r] + pp[r * kD + i];
+  }
+  named_sync(2, 256);
 }
 
 // Work partition: all (stream, tile) pairs in stream order, cut into V equal
@@ -350,6 +359,114 @@ struct SegIter {
   }
 };
 
+// ---------------------------------------------------------------------------
+// Query side of the score MMAs, one CTA of 256 threads per KV stream (runs
+// before the main kernel): q' = RoPE(q), q_rot = Pi_K q', s = S q_rot for the
+// stream's four query rows, then their int8 limbs as the B tiles
+//   B1/B2/B3  rows 4 r + w hold limb w, w-1, w-2 of q_rot row r / sq_r
+//   Bs        rows 4 r + l hold limb l of s'_i = s_i 2^-(i mod 8) / ss_r at K
+//             position 16 (i mod 8) + i / 8
+// (K-major, 128-byte swizzle, 2 KB each) and the row constants scale * sq_r,
+// 2 ss_r and sum_i s_i (sq_r = max|q_rot| / 127, ss_r = max|s'| / 127).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) decode_qprep_kernel(FusedArgs A) {
+  __shared__ __align__(16) float qx[kRows * kD], qr[kRows * kD], sv[kRows * kD], pp[kRows * kD];
+  __shared__ __align__(16) float red[8 * 16];
+  __shared__ __align__(1024) unsigned char bt[4 * 2048];
+  const DecodeArgs& a = A.v;
+  const DecodeShape& sh = a.sh;
+  const int u = threadIdx.x, lane = u & 31;
+  const int64_t bkv = blockIdx.x;
+  const int kv = static_cast<int>(bkv % sh.hkv), bb = static_cast<int>(bkv / sh.hkv);
+  const int G = sh.hq / sh.hkv;
+  auto qrow = [&](int r) -> int64_t { return int64_t(bb) * sh.hq + kv * G + r; };   // nq == 1
+  const bool rope = a.q_pos != nullptr && a.rope_base > 0.0;
+  {
+    const int r = u >> 6, i = u & 63;
+    const int64_t qi = qrow(r) * kD;
+    float x0 = load_elem(a.q, a.q_dtype, qi + i), x1 = load_elem(a.q, a.q_dtype, qi + i + kD / 2);
+    if (rope) {
+      const int pos = a.q_pos[bb];
+      if (pos < 0 && a.d_status) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
+      double sn, cs;
+      sincos(dev::rope_angle(pos, i, kD, a.rope_base), &sn, &cs);
+      const double r0 = double(x0) * cs - double(x1) * sn, r1 = double(x0) * sn + double(x1) * cs;
+      x0 = static_cast<float>(r0);
+      x1 = static_cast<float>(r1);
+    }
+    qx[r * kD + i] = x0;
+    qx[r * kD + i + kD / 2] = x1;
+  }
+  named_sync(2, 256);
+  matvec4_split(a.PiK + int64_t(kv) * a.pi_stride, qx, qr, pp, u);
+  matvec4_split(a.S, qr, sv, pp, u);
+  const int i = u & 127, rr = 2 * (u >> 7);
+  // Row scales: warp w8 covers row w8 / 2, coordinates of half w8 % 2.
+  {
+    const int w8 = u >> 5, r = w8 >> 1, i0 = (w8 & 1) * 64 + lane;
+    float mq = 0.f, ms = 0.f, ssm = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int ii = i0 + 32 * k;
+      const float jsc = __uint_as_float(static_cast<uint32_t>(127 - (ii & 7)) << 23);   // 2^-(i mod 8)
+      mq = fmaxf(mq, fabsf(qr[r * kD + ii]));
+      ms = fmaxf(ms, fabsf(sv[r * kD + ii]) * jsc);
+      ssm += sv[r * kD + ii];
+    }
+    mq = warp_max(mq);
+    ms = warp_max(ms);
+    ssm = warp_sum(ssm);
+    if (lane == 0) {
+      red[w8 * 16 + 0] = mq;
+      red[w8 * 16 + 1] = ms;
+      red[w8 * 16 + 2] = ssm;
+    }
+  }
+  named_sync(2, 256);
+  unsigned char* out = A.qprep + bkv * kQPrepStride;
+  {
+    float sq[2], ss[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int r = rr + k;
+      const float mq = fmaxf(red[(2 * r) * 16 + 0], red[(2 * r + 1) * 16 + 0]);
+      const float ms = fmaxf(red[(2 * r) * 16 + 1], red[(2 * r + 1) * 16 + 1]);
+      sq[k] = mq > 0.f ? mq / 127.f : 1.f;
+      ss[k] = ms > 0.f ? ms / 127.f : 1.f;
+    }
+    if (u < kRows) {
+      const int r = u;
+      const float mq = fmaxf(red[(2 * r) * 16 + 0], red[(2 * r + 1) * 16 + 0]);
+      const float ms = fmaxf(red[(2 * r) * 16 + 1], red[(2 * r + 1) * 16 + 1]);
+      float* qc = reinterpret_cast<float*>(out + 4 * 2048);
+      qc[r] = a.scale * (mq > 0.f ? mq / 127.f : 1.f);
+      qc[4 + r] = 2.f * (ms > 0.f ? ms / 127.f : 1.f);
+      qc[8 + r] = red[(2 * r) * 16 + 2] + red[(2 * r + 1) * 16 + 2];
+      qc[12 + r] = 0.f;
+    }
+    const int ks = 16 * (i & 7) + (i >> 3);
+    const float jsc = __uint_as_float(static_cast<uint32_t>(127 - (i & 7)) << 23);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int r = rr + k;
+      int lq[4], ls[4];
+      limbs4(qr[r * kD + i] / sq[k], lq);
+      limbs4(sv[r * kD + i] * jsc / ss[k], ls);
+#pragma unroll
+      for (int w2 = 0; w2 < 4; ++w2) {
+        bt[sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(lq[w2]));
+        bt[2048 + sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(w2 >= 1 ? lq[w2 - 1] : 0));
+        bt[4096 + sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(w2 >= 2 ? lq[w2 - 2] : 0));
+        bt[6144 + sw_byte(4 * r + w2, ks)] = static_cast<unsigned char>(static_cast<int8_t>(ls[w2]));
+      }
+    }
+  }
+  named_sync(2, 256);
+  // The tiles leave in 16-byte pieces (swizzled layout kept byte for byte).
+#pragma unroll
+  for (int k = 0; k < 2; ++k) reinterpret_cast<uint4*>(out)[u + 256 * k] = reinterpret_cast<const uint4*>(bt)[u + 256 * k];
+}
+
 template <int KB>
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) {
   using Sm = FSm<KB>;
@@ -360,30 +477,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
   const DecodeShape& sh = a.sh;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Sm::kOffBar);
   uint64_t* st_full = bars;                       // [kStages] loader (tx)
-  uint64_t* st_empty = bars + kStages;            // [kStages] 4 key + 4 value warps
-  uint64_t* a_full = bars + 2 * kStages;          // [2] key warps
+  uint64_t* st_empty = bars + kStages;            // [kStages] the tile's key group + value/softmax group
+  uint64_t* a_full = bars + 2 * kStages;          // [2] key group of the buffer
   uint64_t* s_full = a_full + 2;                  // [2] score commit (also frees the A operand)
-  uint64_t* ds_free = s_full + 2;                 // [2] softmax warps read the score columns
-  uint64_t* vh_full = ds_free + 2;                // [2] value warps
-  uint64_t* p_full = vh_full + 2;                 // [2] softmax warps
-  uint64_t* pv_full = p_full + 2;                 // [2] PV commit (frees the value operand and P)
-  uint64_t* bt_full = pv_full + 2;                // [2] per segment parity: the prologue's 8 warps
-  uint64_t* reg_done = bt_full + 2;               // [4] PV commit when a TMEM value region closes
-  uint64_t* reg_free = reg_done + 4;              // [4] value warps folded the region
+  uint64_t* ds_free = s_full + 2;                 // [2] the group read the score columns
+  uint64_t* pv_ready = ds_free + 2;               // [kNVh] the group wrote the value operand and P
+  uint64_t* pv_full = pv_ready + kNVh;            // [kNVh] PV commit (frees the value operand and P)
+  uint64_t* bt_full = pv_full + kNVh;             // [2] per segment parity: the query-side copy (tx)
+  uint64_t* bt_free = bt_full + 2;                // [2] score issuer: the segment's score MMAs are done
+  uint64_t* reg_done = bt_free + 2;               // [4] PV commit when a TMEM value region closes
+  uint64_t* reg_free = reg_done + 4;              // [4] the owning group folded the region
   uint64_t* drain = reg_free + 4;                 // [2] score issuer, PV issuer
   uint64_t* a_free = s_full;
   uint64_t* vh_free = pv_full;
-  uint64_t* p_free = pv_full;
 
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Sm::kOffMisc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + Sm::kOffMisc + 4);
   int* merge_s = reinterpret_cast<int*>(sm + Sm::kOffMisc + 8);
   float* qx = reinterpret_cast<float*>(sm + Sm::kOffQ);             // [4][128] RoPE'd q; merged rows
   float* qr = qx + kRows * kD;                                      // [4][128] q_rot
-  float* sv = qr + kRows * kD;                                      // [4][128] s
   float* red = reinterpret_cast<float*>(sm + Sm::kOffRed);          // [16][16]
-  float* pp = reinterpret_cast<float*>(sm + Sm::kOffPP);            // [3][4][128] partial sums
-  float* segc = reinterpret_cast<float*>(sm + Sm::kOffSeg);         // [2][kSegFloats] per-segment constants
+  float* pp = reinterpret_cast<float*>(sm + Sm::kOffPP);            // [4][128] partial sums
   uint32_t* recs = reinterpret_cast<uint32_t*>(sm + Sm::kOffRec);   // [8][16] tile records
   uint32_t* tab = reinterpret_cast<uint32_t*>(sm + Sm::kOffTab);    // ka1 ka2 ka3 va1 va2 (4 words each)
   float* cb_scale = reinterpret_cast<float*>(sm + Sm::kOffTab + 20 * 4);
@@ -400,11 +514,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       mbar_init(&a_full[b], 4);
       mbar_init(&s_full[b], 1);
       mbar_init(&ds_free[b], 4);
-      mbar_init(&vh_full[b], 4);
-      mbar_init(&p_full[b], 4);
-      mbar_init(&pv_full[b], 1);
-      mbar_init(&bt_full[b], 8);
+
+      mbar_init(&bt_full[b], 1);
+      mbar_init(&bt_free[b], 1);
       mbar_init(&drain[b], 1);
+    }
+    for (int x = 0; x < kNVh; ++x) {
+      mbar_init(&pv_ready[x], 4);
+      mbar_init(&pv_full[x], 1);
     }
     for (int x = 0; x < 4; ++x) {
       mbar_init(&reg_done[x], 1);
@@ -440,6 +557,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       Seg sg;
       while (ok && it.next(sg)) {
         const int64_t row0 = sg.s * sh.ctx_stride;
+        {
+          // The segment's query side (B tiles and row constants) into copy ib,
+          // once the score MMAs of segment idx - 2 are done with it.
+          const int ib = sg.idx & 1;
+          if (*abort_s || !mbar_wait(&bt_free[ib], ((sg.idx >> 1) & 1) ^ 1)) { ok = false; break; }
+          mbar_expect_tx(&bt_full[ib], kQPrepBytes);
+          bulk_g2s(sm + Sm::kOffB + ib * kBStride, A.qprep + sg.s * kQPrepStride, kQPrepBytes, &bt_full[ib]);
+        }
         for (int64_t tt = sg.t0; tt < sg.t1; ++tt, ++j) {
           const int s = j % kStages;
           if (*abort_s || !mbar_wait(&st_empty[s], ((j / kStages) & 1) ^ 1)) { ok = false; break; }
@@ -468,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
     const bool leader = elect_one();
     const uint32_t id_mse = idesc_i8(true, false, false, true), id_sgn = idesc_i8(false, false, false, true);
     const uint32_t id_v = idesc_i8(true, true, true, false);
-    const uint64_t b_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffB));
+    const uint64_t b_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffB));   // copy ib at + ib * kBStride
     const uint64_t vh_desc0 = desc_k_sw128(smem_u32(sm + Sm::kOffVh));
     const uint64_t p_desc0 = desc_mn_noswz(smem_u32(sm + Sm::kOffP));
     int j = 0;
@@ -495,17 +620,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
           const uint32_t a0 = tmem + kColA + b * 128;
           // a1, a2, a3 against B1, B2, B3 (limb-shifted q) into the MSE
           // columns, the sign chunk into its own columns.
-          const uint64_t bs = b_desc0 + (((ib * 4 + 3) * 2048) >> 4);
+          const uint64_t bs = b_desc0 + ((ib * kBStride + 3 * 2048) >> 4);
 #pragma unroll
           for (int step = 0; step < 12; ++step) {
             const int ch = step >> 2, k = step & 3;
-            const uint64_t bq = b_desc0 + (((ib * 4 + ch) * 2048) >> 4);
+            const uint64_t bq = b_desc0 + ((ib * kBStride + ch * 2048) >> 4);
             if (leader) umma_i8_ts(d, a0 + ch * 32 + k * 8, bq + ((k * 32) >> 4), id_mse, step != 0);
             if (step < 4 && leader) umma_i8_ts(d + 16, a0 + 96 + k * 8, bs + ((k * 32) >> 4), id_sgn, k != 0);
           }
-          if (leader) umma_commit(&s_full[b]);
+          if (leader) {
+            umma_commit(&s_full[b]);
+            if (tj == nt_tiles - 1) umma_commit(&bt_free[ib]);   // the query-side copy is free
+          }
         } else {
-          const bool w = mbar_wait(&vh_full[b], ph) && mbar_wait(&p_full[b], ph);
+          const int xb = j % kNVh;                  // value operand / P buffer of the tile
+          const bool w = mbar_wait(&pv_ready[xb], (j / kNVh) & 1);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           tc_fence_after();
           const bool flip = recs[(j & 7) * 16 + 1] != 0u;
@@ -526,16 +655,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
               !__all_sync(0xffffffffu, mbar_wait(&reg_free[X], (nclose - 1) & 1))) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + kColDo + X * 32;
-          const uint64_t pb = p_desc0 + ((b * 2048) >> 4);
+          const uint64_t pb = p_desc0 + ((xb * 2048) >> 4);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {             // 32 tokens per step = 4 atoms of 8 tokens
 #pragma unroll
             for (int limb = 0; limb < 2; ++limb) {  // the two limb chains alternate
-              const uint64_t ad = vh_desc0 + ((b * Sm::kVhBytes + limb * kTT * 128 + k * 4096) >> 4);
+              const uint64_t ad = vh_desc0 + ((xb * Sm::kVhBytes + limb * kTT * 128 + k * 4096) >> 4);
               if (leader) umma_i8_ss(d + limb * 16, ad, pb + ((k * 512) >> 4), id_v, !(fresh && k == 0));
             }
           }
-          if (leader) umma_commit(&pv_full[b]);
+          if (leader) umma_commit(&pv_full[xb]);
           if (tj >= nt_tiles - 2) {
             // The group's last tile of the segment: close its region; its next
             // segment starts in the other one.
@@ -552,8 +681,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
     if (leader) umma_commit(&drain[warp == kWScore ? 0 : 1]);
     __syncwarp();
     mbar_wait(&drain[warp == kWScore ? 0 : 1], 0);
-  } else if (warp >= kWKey0 && warp < kWKey0 + 4) {
-    // ------------------------------------------------- key operands (TMEM)
+  } else if (warp >= kWKey0 && warp < kWVs0) {
+    // ---------------------------------- key operands (TMEM), two groups of 4 warps
+    // Key group kg builds the A operand of the tiles with j % 2 == kg (its
+    // own TMEM buffer).
+    const int kg = (warp - kWKey0) >> 2;
     const int q = warp & 3;                       // lane quadrant
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int row = q * 32 + lane;                // token = TMEM lane this thread writes
@@ -573,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
         const int s = j % kStages;
         const int b = j & 1;
+        if (b != kg) continue;
         if (!__all_sync(0xffffffffu, mbar_wait(&st_full[s], (j / kStages) & 1))) {
           if (lane == 0) fail();
           stop = true;
@@ -643,17 +776,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
         if (lane == 0) mbar_arrive(&a_full[b]);
       }
     }
-  } else if (warp >= kWVal0) {
-    // ------------------------------------------ value warps and softmax warps
-    // The value group and both softmax groups share the per-segment prologue
-    // and the combine's arrival (384 threads on barrier 2); then each runs its
-    // own per-tile loop. Softmax group g takes the segment's tiles tj with
-    // tj % 2 == g and keeps its own running maxima, sums and TMEM regions
-    // (2g, 2g + 1), so the two groups' per-tile chains overlap.
-    const bool is_val = warp < kWSoft0;
-    const int sgrp = is_val ? -1 : (warp - kWSoft0) >> 2;   // softmax group
-    const int sbar = sgrp == 0 ? 1 : 4;                       // its named barrier (128 threads)
-    const int u = tid - kWVal0 * 32;              // 0..383; the prologue's work is on u < 256
+  } else if (warp >= kWVs0) {
+    // ---------------------------------------- value + softmax groups (2 x 4 warps)
+    // Group g takes the segment's tiles tj with tj % 2 == g: it builds the
+    // tile's value operand, turns its scores into weights and folds its own
+    // TMEM regions (2g, 2g + 1). Both groups share the segment prologue, the
+    // arrival and the combine (256 threads on barrier 2).
+    const int grp = (warp - kWVs0) >> 2;          // 0 or 1
+    const int gbar = grp == 0 ? 1 : 4;            // the group's named barrier (128 threads)
+    const int u = tid - kWVs0 * 32;               // 0..255
     const int q = warp & 3;                       // lane quadrant
     const int lrow = q * 32 + lane;               // token (TMEM lane) / coordinate
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -662,9 +793,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
     const uint32_t v1t[2] = {tab[12], tab[13]}, v2t[2] = {tab[16], tab[17]};
     int j = 0;                                    // CTA-local tile counter
     bool stop = false;
-    // value warps: TMEM region bookkeeping (mirrors the PV issuer)
-    int vcur[2] = {0, 0};
-    int closes[4] = {0, 0, 0, 0};
+    uint32_t gcur = 0u;                           // region in use: 2 grp + gcur
+    uint32_t gcl = 0u;                            // closes of the group's two regions (byte each)
+    float* nring = reinterpret_cast<float*>(sm + Sm::kOffNrm) + grp * (4 * 3 * kTT);
     SegIter it(part);
     Seg sg;
     while (it.next(sg)) {
@@ -674,15 +805,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       const int kv = static_cast<int>(bkv % sh.hkv), bb = static_cast<int>(bkv / sh.hkv);
       const int64_t row0 = bkv * sh.ctx_stride;
       const int64_t te = (sg.t1 * kTT < sh.n_ctx ? sg.t1 * kTT : sh.n_ctx);
-      const int64_t rec_idx = sg.v + sg.s;
       const int j0 = j;
       auto qrow = [&](int r) -> int64_t { return int64_t(bb) * sh.hq + kv * G + r; };   // nq == 1
-      float* segk = segc + ib * kSegFloats;
-      // Softmax group: norms of its k-th tile (tile 2k + g) go into ring slot
-      // k % 4, three tiles ahead, by cp.async (one commit group per tile).
-      float* nring = reinterpret_cast<float*>(sm + Sm::kOffNrm) + (sgrp < 0 ? 0 : sgrp) * (4 * 3 * kTT);
+      // Norms of the group's k-th tile (tile 2k + grp) go into ring slot k % 4,
+      // three tiles ahead, by cp.async (one commit group per tile).
       auto norm_fetch = [&](int k) {
-        const int tj = 2 * k + sgrp;
+        const int tj = 2 * k + grp;
         if (tj < nt_tiles) {
           const int64_t t = (sg.t0 + tj) * kTT + lrow;
           const bool ok = t < te;
@@ -695,188 +823,198 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
         }
         cp_async_commit();
       };
-      if (!is_val) {
-        norm_fetch(0);
-        norm_fetch(1);
-        norm_fetch(2);
+      norm_fetch(0);
+      norm_fetch(1);
+      norm_fetch(2);
+      // ---------------- the segment's query side (copied in by the loader)
+      if (!__all_sync(0xffffffffu, mbar_wait(&bt_full[ib], (sg.idx >> 1) & 1)) && lane == 0) fail();
+      const float* qc = reinterpret_cast<const float*>(sm + Sm::kOffB + ib * kBStride + 4 * 2048);
+      // ---------------- the group's tiles
+      float kq[kRows], ks2[kRows], ssum[kRows];
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        kq[r] = qc[r] * k_scale;
+        ks2[r] = qc[4 + r];
+        ssum[r] = qc[8 + r];
       }
-      // ---------------- prologue: q_rot = Pi_K RoPE(q), s = S q_rot, B tiles
-      {
-        const bool work = u < 256;
-        const bool rope = a.q_pos != nullptr && a.rope_base > 0.0;
-        if (work) {
-          const int r = u >> 6, i = u & 63;
-          const int64_t qi = qrow(r) * kD;
-          float x0 = load_elem(a.q, a.q_dtype, qi + i), x1 = load_elem(a.q, a.q_dtype, qi + i + kD / 2);
-          if (rope) {
-            const int pos = a.q_pos[bb];
-            if (pos < 0 && a.d_status) atomicOr(a.d_status, TQ_DEV_BAD_POSITION);
-            double sn, cs;
-            sincos(dev::rope_angle(pos, i, kD, a.rope_base), &sn, &cs);
-            const double r0 = double(x0) * cs - double(x1) * sn, r1 = double(x0) * sn + double(x1) * cs;
-            x0 = static_cast<float>(r0);
-            x1 = static_cast<float>(r1);
-          }
-          qx[r * kD + i] = x0;
-          qx[r * kD + i + kD / 2] = x1;
-        }
-        named_sync(2, 384);
-        const int i = u & 127, rr = 2 * ((u >> 7) & 1);
-        // q_rot = Pi_K qx, then s = S q_rot.
-        matvec4_split(a.PiK + int64_t(kv) * a.pi_stride, qx, qr, pp, u);
-        matvec4_split(a.S, qr, sv, pp, u);
-        // Row scales: warp w8 = u / 32 covers row w8 / 2, coordinates of half w8 % 2.
-        if (work) {
-          const int w8 = u >> 5, r = w8 >> 1, i0 = (w8 & 1) * 64 + lane;
-          float mq = 0.f, ms = 0.f, ssm = 0.f;
+      const float kr = a.scale * alpha;
+      float m_run[kRows], l_part[kRows], acc[kRows], m_acc[kRows];
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int ii = i0 + 32 * k;
-            const float jsc = __uint_as_float(static_cast<uint32_t>(127 - (ii & 7)) << 23);   // 2^-(i mod 8)
-            mq = fmaxf(mq, fabsf(qr[r * kD + ii]));
-            ms = fmaxf(ms, fabsf(sv[r * kD + ii]) * jsc);
-            ssm += sv[r * kD + ii];
-          }
-          mq = warp_max(mq);
-          ms = warp_max(ms);
-          ssm = warp_sum(ssm);
-          if (lane == 0) {
-            red[w8 * 16 + 0] = mq;
-            red[w8 * 16 + 1] = ms;
-            red[w8 * 16 + 2] = ssm;
-          }
-        }
-        named_sync(2, 384);
-        if (work) {
-          float sq[2], ss[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int r = rr + k;
-            const float mq = fmaxf(red[(2 * r) * 16 + 0], red[(2 * r + 1) * 16 + 0]);
-            const float ms = fmaxf(red[(2 * r) * 16 + 1], red[(2 * r + 1) * 16 + 1]);
-            sq[k] = mq > 0.f ? mq / 127.f : 1.f;
-            ss[k] = ms > 0.f ? ms / 127.f : 1.f;
-          }
-          if (u < kRows) {
-            const int r = u;
-            const float mq = fmaxf(red[(2 * r) * 16 + 0], red[(2 * r + 1) * 16 + 0]);
-            const float ms = fmaxf(red[(2 * r) * 16 + 1], red[(2 * r + 1) * 16 + 1]);
-            const float sqr = mq > 0.f ? mq / 127.f : 1.f, ssr = ms > 0.f ? ms / 127.f : 1.f;
-            segk[r] = a.scale * k_scale * sqr;                                   // mse scale
-            segk[4 + r] = 2.f * ssr;                                             // sign-sum scale
-            segk[8 + r] = red[(2 * r) * 16 + 2] + red[(2 * r + 1) * 16 + 2];     // sum s
-          }
-          // B tiles: B1/B2/B3 rows 4 r + w hold limb w, w-1, w-2 of q_rot row r;
-          // Bs rows 4 r + l hold limb l of s' at K position 16 (i mod 8) + i / 8.
-          unsigned char* bt = sm + Sm::kOffB + ib * 4 * 2048;
-          const int ks = 16 * (i & 7) + (i >> 3);
-          const float jsc = __uint_as_float(static_cast<uint32_t>(127 - (i & 7)) << 23);
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int r = rr + k;
-            int lq[4], ls[4];
-            limbs4(qr[r * kD + i] / sq[k], lq);
-            limbs4(sv[r * kD + i] * jsc / ss[k], ls);
-#pragma unroll
-            for (int w2 = 0; w2 < 4; ++w2) {
-              bt[sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(lq[w2]));
-              bt[2048 + sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(w2 >= 1 ? lq[w2 - 1] : 0));
-              bt[4096 + sw_byte(4 * r + w2, i)] = static_cast<unsigned char>(static_cast<int8_t>(w2 >= 2 ? lq[w2 - 2] : 0));
-              bt[6144 + sw_byte(4 * r + w2, ks)] = static_cast<unsigned char>(static_cast<int8_t>(ls[w2]));
-            }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bt_full[ib]);
-        }
-        named_sync(2, 384);     // segk visible to all groups; qx/qr/sv free again
+      for (int r = 0; r < kRows; ++r) {
+        m_run[r] = -INFINITY;
+        l_part[r] = 0.f;
+        acc[r] = 0.f;
+        m_acc[r] = -INFINITY;
       }
-      if (is_val) {
-        // ------------------------------------------------ value warps
-        const int crd = lrow;                     // coordinate (fold, combine)
-        float acc[2][kRows], m_acc[2][kRows];
+      float v0 = 0.f, inv_v0 = 0.f;
+      // Folds the group's current region (closed by the PV issuer; running
+      // maxima m_seg in effect for its tiles) into acc (thread = coordinate),
+      // then moves to the other region.
+      auto fold = [&](const float (&m_seg)[kRows]) -> bool {
+        const int X = 2 * grp + static_cast<int>(gcur);
+        const uint32_t nclose = (gcl >> (8 * gcur)) & 0xFFu;
+        if (!__all_sync(0xffffffffu, mbar_wait(&reg_done[X], nclose & 1))) return false;
+        tc_fence_after();
+        uint32_t dv[32];
+        tmem_ld32(lane_addr + kColDo + X * 32, dv);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&reg_free[X]);
+        gcl += 1u << (8 * gcur);
+        gcur ^= 1u;
 #pragma unroll
-        for (int g = 0; g < 2; ++g)
+        for (int r = 0; r < kRows; ++r) {
+          float w0 = 0.f, w1 = 0.f;
 #pragma unroll
-          for (int r = 0; r < kRows; ++r) {
-            acc[g][r] = 0.f;
-            m_acc[g][r] = -INFINITY;
+          for (int w8 = 3; w8 >= 0; --w8) {
+            w0 = fmaf(w0, 256.f, static_cast<float>(static_cast<int32_t>(dv[4 * r + w8])));
+            w1 = fmaf(w1, 256.f, static_cast<float>(static_cast<int32_t>(dv[16 + 4 * r + w8])));
           }
-        // Folds group g's current TMEM region (closed; running maxima m_seg in
-        // effect for its tiles) into the registers, then moves to the other.
-        auto fold = [&](int g, const float (&m_seg)[kRows]) -> bool {
-          const int X = 2 * g + vcur[g];
-          if (!__all_sync(0xffffffffu, mbar_wait(&reg_done[X], closes[X] & 1))) return false;
-          tc_fence_after();
-          uint32_t dv[32];
-          tmem_ld32(lane_addr + kColDo + X * 32, dv);
+          const float val = v_scale * fmaf(w1, 1.f / 128.f, w0) * (1.f / 16777216.f);
+          const float c = (m_acc[r] == -INFINITY) ? 0.f : ex2(m_acc[r] - m_seg[r]);
+          acc[r] = fmaf(acc[r], c, val);
+          m_acc[r] = m_seg[r];
+        }
+        return true;
+      };
+      for (int k = 0; 2 * k + grp < nt_tiles; ++k) {
+        const int tj = 2 * k + grp;
+        const int jt = j0 + tj;
+        const int b = jt & 1, s = jt % kStages;
+        const int64_t t0 = (sg.t0 + tj) * kTT;
+        const int nt = static_cast<int>((sh.n_ctx - t0 < kTT ? sh.n_ctx - t0 : int64_t(kTT)));
+        const bool valid = lrow < nt;
+        norm_fetch(k + 3);
+        // -- scores of the tile (thread = token)
+        cp_async_wait<3>();
+        const float* slot = nring + (k & 3) * (3 * kTT);
+        const float kn = slot[lrow], rn = slot[kTT + lrow], vn = slot[2 * kTT + lrow];
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (jt >> 1) & 1));
+        tc_fence_after();
+        // MSE part: weights 1, 1/128, 1/128^2 of the key-limb products
+        // (weight 3 is below 1e-6 of the first); sign part: four limbs.
+        // The two halves are read one after the other (fewer live registers).
+        float mse[kRows], sgn[kRows];
+        {
+          uint32_t d[16];
+          tmem_ld16(lane_addr + kColDs + b * 32, d);
           tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&reg_free[X]);
-          ++closes[X];
-          vcur[g] ^= 1;
 #pragma unroll
           for (int r = 0; r < kRows; ++r) {
-            float v0 = 0.f, v1 = 0.f;
+            const int32_t m01 = static_cast<int32_t>(d[4 * r]) * 128 + static_cast<int32_t>(d[4 * r + 1]);
+            mse[r] = fmaf(static_cast<float>(static_cast<int32_t>(d[4 * r + 2])), 1.f / 16384.f,
+                          static_cast<float>(m01) * (1.f / 128.f));
+          }
+          tmem_ld16(lane_addr + kColDs + b * 32 + 16, d);
+          tmem_ld_wait();
 #pragma unroll
-            for (int w8 = 3; w8 >= 0; --w8) {
-              v0 = fmaf(v0, 256.f, static_cast<float>(static_cast<int32_t>(dv[4 * r + w8])));
-              v1 = fmaf(v1, 256.f, static_cast<float>(static_cast<int32_t>(dv[16 + 4 * r + w8])));
-            }
-            const float val = v_scale * fmaf(v1, 1.f / 128.f, v0) * (1.f / 16777216.f);
-            const float c = (m_acc[g][r] == -INFINITY) ? 0.f : ex2(m_acc[g][r] - m_seg[r]);
-            acc[g][r] = fmaf(acc[g][r], c, val);
-            m_acc[g][r] = m_seg[r];
+          for (int r = 0; r < kRows; ++r) {
+            const int32_t e01 = static_cast<int32_t>(d[4 * r]) * 128 + static_cast<int32_t>(d[4 * r + 1]);
+            const int32_t e23 = static_cast<int32_t>(d[4 * r + 2]) * 128 + static_cast<int32_t>(d[4 * r + 3]);
+            sgn[r] = fmaf(static_cast<float>(e23), 1.f / 2097152.f, static_cast<float>(e01) * (1.f / 128.f));
           }
-          return true;
-        };
-        // Waits for the record of tile jj (CTA-local index).
-        auto rec_ready = [&](int jj) -> bool {
-          volatile uint32_t* rc = recs + (jj & 7) * 16;
-          bool ok = rc[0] == static_cast<uint32_t>(jj);
-          if (!ok) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!(ok = (rc[0] == static_cast<uint32_t>(jj))) && globaltimer_ns() - t0 < 2000000000ull) {
-            }
-          }
-          const bool all = __all_sync(0xffffffffu, ok);
-          __threadfence_block();
-          return all;
-        };
-        // Reads the softmax's record of tile jj; folds the region it closed.
-        auto take_rec = [&](int jj) -> bool {
-          if (!rec_ready(jj)) return false;
-          volatile uint32_t* rc = recs + (jj & 7) * 16;
-          if (rc[1] != 0u) {
-            float mo[kRows];
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_free[b]);
+        float s2[kRows];
 #pragma unroll
-            for (int r = 0; r < kRows; ++r) mo[r] = __uint_as_float(rc[2 + r]);
-            if (!fold((jj - j0) & 1, mo)) return false;
+        for (int r = 0; r < kRows; ++r) {
+          const float qjl = fmaf(ks2[r], sgn[r], -ssum[r]);
+          const float sn = fmaf(kq[r] * kn, mse[r], kr * rn * qjl);
+          if (a.scores_out && valid) a.scores_out[qrow(r) * sh.n_ctx + t0 + lrow] = sn;
+          s2[r] = valid ? sn * kLog2e : -INFINITY;
+        }
+        bool flip = false;
+        float m_old[kRows];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) m_old[r] = m_run[r];
+        float x[kRows], p[kRows];
+        if (k == 0) {
+          // The group's first tile sets its running maxima and V0.
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            const float mx = warp_max(s2[r]);
+            if (lane == 0) red[(8 + 4 * grp + q) * 16 + r] = mx;
           }
-          return true;
-        };
-        for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
-          const int s = j % kStages;
-          const int b = j & 1;
-          const int row = lrow;                   // token within the tile (operands)
-          if (!__all_sync(0xffffffffu, mbar_wait(&st_full[s], (j / kStages) & 1))) {
-            if (lane == 0) fail();
+          {
+            const float vm = warp_max(valid ? vn : 0.f);
+            if (lane == 0) red[(8 + 4 * grp + q) * 16 + 4] = vm;
+          }
+          named_sync(gbar, 128);
+          v0 = 0.f;
+#pragma unroll
+          for (int w2 = 0; w2 < 4; ++w2) v0 = fmaxf(v0, red[(8 + 4 * grp + w2) * 16 + 4]);
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            float mx = red[(8 + 4 * grp) * 16 + r];
+#pragma unroll
+            for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, red[(8 + 4 * grp + w2) * 16 + r]);
+            m_run[r] = mx;
+            m_old[r] = mx;
+          }
+          inv_v0 = v0 > 0.f ? 1.f / v0 : 0.f;
+          named_sync(gbar, 128);
+        }
+        const float wv = vn * inv_v0;
+        bool need = false;
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          p[r] = valid ? ex2(fminf(s2[r] - m_run[r], 100.f)) : 0.f;
+          x[r] = p[r] * wv;
+          need |= !(x[r] <= 64.f) && valid;
+        }
+        // One vote per tile (uniform over the group's four warps): a weight
+        // out of range, or a failed wait / abort anywhere in the group.
+        const bool bad = !ok || *abort_s != 0;
+        if (wg_sync_or(gbar, need || bad)) {
+          if (wg_sync_or(gbar, bad)) {
+            if (!ok && lane == 0) fail();
             stop = true;
             break;
           }
-          const unsigned char* st = sm + s * Sm::kStageStride;
-          const uint32_t* wrow = reinterpret_cast<const uint32_t*>(st + Sm::kOffVi + row * 48);
-          if (!__all_sync(0xffffffffu, mbar_wait(&vh_free[b], ((j >> 1) & 1) ^ 1))) {
-            if (lane == 0) fail();
-            stop = true;
-            break;
+          // A weight would leave the fixed-point range: move the running
+          // maximum by the whole number of octaves that brings every weight
+          // of the tile back to <= 1.
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            const float z = valid ? (s2[r] - m_run[r]) + __log2f(fmaxf(wv, 1e-30f)) : -INFINITY;
+            const float zm = warp_max(z);
+            if (lane == 0) red[(8 + 4 * grp + q) * 16 + r] = zm;
           }
-          unsigned char* vh = sm + Sm::kOffVh + b * Sm::kVhBytes;
-          // Row `row` (token) of each limb tile: 128 coordinate bytes, M-major,
-          // 8-token atoms of 1024 bytes. 32 coordinates (12 code bytes, w[0..2])
-          // per iteration; the words shift down after each one.
-          const int atom = row >> 3, r8 = row & 7;
+          named_sync(gbar, 128);
+#pragma unroll
+          for (int r = 0; r < kRows; ++r) {
+            float zm = red[(8 + 4 * grp) * 16 + r];
+#pragma unroll
+            for (int w2 = 1; w2 < 4; ++w2) zm = fmaxf(zm, red[(8 + 4 * grp + w2) * 16 + r]);
+            const float dl = zm > 0.f ? ceilf(zm) : 0.f;
+            m_run[r] += dl;
+            l_part[r] *= ex2(-dl);
+            p[r] = valid ? ex2(s2[r] - m_run[r]) : 0.f;
+            x[r] = p[r] * wv;
+          }
+          named_sync(gbar, 128);
+          flip = true;
+        }
+        uint32_t X[kRows];
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          l_part[r] += p[r];
+          X[r] = valid ? __float2uint_rn(x[r] * 16777216.f) : 0u;
+        }
+        // -- value operand of the tile (thread = token): two int8 limbs of the
+        // value codebook, one 128-byte M-major row per token and limb.
+        // (Built after the scores: the buffer, xb = jt % 3, is freed by the
+        // product of tile jt - 3, which is usually done by now.)
+        const int xb = jt % kNVh;
+        const bool okv = mbar_wait(&st_full[s], (jt / kStages) & 1) && mbar_wait(&vh_free[xb], ((jt / kNVh) & 1) ^ 1);
+        if (!__all_sync(0xffffffffu, okv) && lane == 0) fail();
+        {
+          const uint32_t* wrow = reinterpret_cast<const uint32_t*>(sm + s * Sm::kStageStride + Sm::kOffVi + lrow * 48);
+          unsigned char* vh = sm + Sm::kOffVh + xb * Sm::kVhBytes;
+          const int atom = lrow >> 3, r8 = lrow & 7;
 #pragma unroll 1
           for (int c2 = 0; c2 < 4; ++c2) {
             const uint32_t x4[4] = {wrow[3 * c2], wrow[3 * c2 + 1], wrow[3 * c2 + 2], 0u};
@@ -900,248 +1038,66 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
               *reinterpret_cast<uint4*>(vh + kTT * 128 + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
             }
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&st_empty[s]);
-            mbar_arrive(&vh_full[b]);
-          }
-          // The softmax of tile j - 2 is done (its PV product freed this buffer).
-          if (tj >= 2 && !take_rec(j - 2)) {
-            if (lane == 0) fail();
-            stop = true;
-            break;
-          }
         }
-        // Segment end: the last tiles' records, then each group's final region.
-        bool okr = !stop;
-        for (int jj = max(j0, j - 2); jj < j && okr; ++jj) okr = take_rec(jj);
-        bool ran[2] = {false, false};
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          if (!okr || nt_tiles <= g) continue;
-          const int last = j0 + nt_tiles - 1 - ((nt_tiles - 1 - g) & 1);   // the group's last tile
-          float mf[kRows];
-          {
-            volatile uint32_t* rc = recs + (last & 7) * 16;
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) mf[r] = __uint_as_float(rc[6 + r]);
-          }
-          if (!fold(g, mf)) okr = false;
-          ran[g] = true;     // acc[g] is now relative to the group's final maxima
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&st_empty[s]);
+        *reinterpret_cast<uint4*>(sm + Sm::kOffP + xb * 2048 + lrow * 16) = make_uint4(X[0], X[1], X[2], X[3]);
+        if (lrow == 0) recs[(jt & 7) * 16 + 1] = flip ? 1u : 0u;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pv_ready[xb]);
+        // The PV issuer closes the group's region before this tile's product;
+        // fold it now (rare).
+        if (flip && !fold(m_old)) {
+          if (lane == 0) fail();
         }
-        if (!okr) {
+      }
+      cp_async_wait<0>();
+      j = j0 + nt_tiles;
+      // -------- segment end: the group's final region; its partial record
+      // (v + s) * 2 + grp holds m, l and the rotated output sum.
+      const int64_t rec = (sg.v + sg.s) * 2 + grp;
+      if (nt_tiles > grp) {
+        if (!stop && !fold(m_run)) {
           if (lane == 0) fail();
           stop = true;
         }
-        // Partial record: both groups' sums on the larger of their maxima.
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          float o = 0.f;
-          const float M = ran[1] ? fmaxf(m_acc[0][r], m_acc[1][r]) : m_acc[0][r];
-          if (ran[0]) o = acc[0][r] * segk[16] * ex2(m_acc[0][r] - M);
-          if (ran[1]) o = fmaf(acc[1][r] * segk[17], ex2(m_acc[1][r] - M), o);
-          a.part[(rec_idx * kRows + r) * kRecFloats + crd] = o;
-        }
-      } else {
-        // ---------------------------------------------- softmax group sgrp
-        float kq[kRows], ks2[kRows], ssum[kRows];
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          kq[r] = segk[r];
-          ks2[r] = segk[4 + r];
-          ssum[r] = segk[8 + r];
-        }
-        const float kr = a.scale * alpha;
-        float m_run[kRows], l_part[kRows];
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          m_run[r] = -INFINITY;
-          l_part[r] = 0.f;
-        }
-        float inv_v0 = 0.f;
-        for (int k = 0; 2 * k + sgrp < nt_tiles; ++k) {
-          const int tj = 2 * k + sgrp;
-          const int jt = j0 + tj;
-          const int b = jt & 1;
-          const int64_t t0 = (sg.t0 + tj) * kTT;
-          const int nt = static_cast<int>((sh.n_ctx - t0 < kTT ? sh.n_ctx - t0 : int64_t(kTT)));
-          const bool valid = lrow < nt;
-          norm_fetch(k + 3);
-          cp_async_wait<3>();
-          const float* slot = nring + (k & 3) * (3 * kTT);
-          const float kn = slot[lrow], rn = slot[kTT + lrow], vn = slot[2 * kTT + lrow];
-          const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (jt >> 1) & 1));
-          tc_fence_after();
-          // MSE part: weights 1, 1/128, 1/128^2 of the key-limb products
-          // (weight 3 is below 1e-6 of the first); sign part: four limbs.
-          // The two halves are read one after the other (fewer live registers).
-          float mse[kRows], sgn[kRows];
-          {
-            uint32_t d[16];
-            tmem_ld16(lane_addr + kColDs + b * 32, d);
-            tmem_ld_wait();
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              const int32_t m01 = static_cast<int32_t>(d[4 * r]) * 128 + static_cast<int32_t>(d[4 * r + 1]);
-              mse[r] = fmaf(static_cast<float>(static_cast<int32_t>(d[4 * r + 2])), 1.f / 16384.f,
-                            static_cast<float>(m01) * (1.f / 128.f));
-            }
-            tmem_ld16(lane_addr + kColDs + b * 32 + 16, d);
-            tmem_ld_wait();
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              const int32_t e01 = static_cast<int32_t>(d[4 * r]) * 128 + static_cast<int32_t>(d[4 * r + 1]);
-              const int32_t e23 = static_cast<int32_t>(d[4 * r + 2]) * 128 + static_cast<int32_t>(d[4 * r + 3]);
-              sgn[r] = fmaf(static_cast<float>(e23), 1.f / 2097152.f, static_cast<float>(e01) * (1.f / 128.f));
-            }
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ds_free[b]);
-          float s2[kRows];
-#pragma unroll
-          for (int r = 0; r < kRows; ++r) {
-            const float qjl = fmaf(ks2[r], sgn[r], -ssum[r]);
-            const float mse_r = mse[r];
-            const float sn = fmaf(kq[r] * kn, mse_r, kr * rn * qjl);
-            if (a.scores_out && valid) a.scores_out[qrow(r) * sh.n_ctx + t0 + lrow] = sn;
-            s2[r] = valid ? sn * kLog2e : -INFINITY;
-          }
-          bool flip = false;
-          float m_old[kRows];
-#pragma unroll
-          for (int r = 0; r < kRows; ++r) m_old[r] = m_run[r];
-          float x[kRows], p[kRows];
-          if (k == 0) {
-            // The group's first tile sets its running maxima and V0.
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              const float mx = warp_max(s2[r]);
-              if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + r] = mx;
-            }
-            {
-              const float vm = warp_max(valid ? vn : 0.f);
-              if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + 4] = vm;
-            }
-            named_sync(sbar, 128);
-            float v0 = 0.f;
-#pragma unroll
-            for (int w2 = 0; w2 < 4; ++w2) v0 = fmaxf(v0, red[(8 + 4 * sgrp + w2) * 16 + 4]);
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              float mx = red[(8 + 4 * sgrp) * 16 + r];
-#pragma unroll
-              for (int w2 = 1; w2 < 4; ++w2) mx = fmaxf(mx, red[(8 + 4 * sgrp + w2) * 16 + r]);
-              m_run[r] = mx;
-              m_old[r] = mx;
-            }
-            inv_v0 = v0 > 0.f ? 1.f / v0 : 0.f;
-            if (lrow == 0) segk[16 + sgrp] = v0;
-            named_sync(sbar, 128);
-          }
-          const float wv = vn * inv_v0;
-          bool need = false;
-#pragma unroll
-          for (int r = 0; r < kRows; ++r) {
-            p[r] = valid ? ex2(fminf(s2[r] - m_run[r], 100.f)) : 0.f;
-            x[r] = p[r] * wv;
-            need |= !(x[r] <= 64.f) && valid;
-          }
-          // One vote per tile (uniform over the group's four warps): a weight
-          // out of range, or a failed wait / abort anywhere in the group.
-          const bool bad = !ok || *abort_s != 0;
-          if (wg_sync_or(sbar, need || bad)) {
-            if (wg_sync_or(sbar, bad)) {
-              if (!ok && lane == 0) fail();
-              stop = true;
-              break;
-            }
-            // A weight would leave the fixed-point range: move the running
-            // maximum by the whole number of octaves that brings every weight
-            // of the tile back to <= 1.
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              const float z = valid ? (s2[r] - m_run[r]) + __log2f(fmaxf(wv, 1e-30f)) : -INFINITY;
-              const float zm = warp_max(z);
-              if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + r] = zm;
-            }
-            named_sync(sbar, 128);
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              float zm = red[(8 + 4 * sgrp) * 16 + r];
-#pragma unroll
-              for (int w2 = 1; w2 < 4; ++w2) zm = fmaxf(zm, red[(8 + 4 * sgrp + w2) * 16 + r]);
-              const float dl = zm > 0.f ? ceilf(zm) : 0.f;
-              m_run[r] += dl;
-              l_part[r] *= ex2(-dl);
-              p[r] = valid ? ex2(s2[r] - m_run[r]) : 0.f;
-              x[r] = p[r] * wv;
-            }
-            named_sync(sbar, 128);
-            flip = true;
-          }
-          uint32_t X[kRows];
-#pragma unroll
-          for (int r = 0; r < kRows; ++r) {
-            l_part[r] += p[r];
-            X[r] = valid ? __float2uint_rn(x[r] * 16777216.f) : 0u;
-          }
-          if (!__all_sync(0xffffffffu, mbar_wait(&p_free[b], ((jt >> 1) & 1) ^ 1)) && lane == 0) fail();
-          *reinterpret_cast<uint4*>(sm + Sm::kOffP + b * 2048 + lrow * 16) = make_uint4(X[0], X[1], X[2], X[3]);
-          if (lrow == 0) {
-            volatile uint32_t* rc = recs + (jt & 7) * 16;
-            rc[1] = flip ? 1u : 0u;
-#pragma unroll
-            for (int r = 0; r < kRows; ++r) {
-              rc[2 + r] = __float_as_uint(m_old[r]);
-              rc[6 + r] = __float_as_uint(m_run[r]);
-            }
-            __threadfence_block();
-            rc[0] = static_cast<uint32_t>(jt);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&p_full[b]);
-        }
-        cp_async_wait<0>();
-        j = j0 + nt_tiles;
-        // Segment end: the group's l per row; its m and l for the record (the
-        // four warps stopped together or not at all).
         if (!stop) {
 #pragma unroll
           for (int r = 0; r < kRows; ++r) {
             const float x = warp_sum(l_part[r]);
-            if (lane == 0) red[(8 + 4 * sgrp + q) * 16 + 8 + r] = x;
+            if (lane == 0) red[(8 + 4 * grp + q) * 16 + 8 + r] = x;
           }
-          named_sync(sbar, 128);
-          if (lrow < kRows) {
-            const int r = lrow;
-            const float* rg = red + (8 + 4 * sgrp) * 16 + 8 + r;
-            segk[20 + 8 * sgrp + r] = m_run[r];
-            segk[24 + 8 * sgrp + r] = rg[0] + rg[16] + rg[32] + rg[48];
+        }
+        named_sync(gbar, 128);
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          float* pr = a.part + (rec * kRows + r) * kRecFloats;
+          pr[lrow] = acc[r] * v0;
+          if (lrow == 0) {
+            const float* rg = red + (8 + 4 * grp) * 16 + 8 + r;
+            pr[kD] = m_run[r];
+            pr[kD + 1] = rg[0] + rg[16] + rg[32] + rg[48];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          float* pr = a.part + (rec * kRows + r) * kRecFloats;
+          pr[lrow] = 0.f;
+          if (lrow == 0) {
+            pr[kD] = -INFINITY;
+            pr[kD + 1] = 0.f;
           }
         }
       }
-      // ---------------- arrival; the stream's last segment merges. All groups
+      // ---------------- arrival; the stream's last segment merges. Both groups
       // pass the same barriers whether or not they stopped; the decision to
       // quit is taken once, after the first of them.
       __threadfence();
-      named_sync(2, 384);
+      named_sync(2, 256);
       if (u == 0) {
         merge_s[1] = *abort_s != 0 ? 1 : 0;
-        // m and l of the segment's record from the two groups' (a group
-        // without tiles has m = -inf, l = 0).
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) {
-          const float m0 = segk[20 + r], l0 = segk[24 + r];
-          const float m1 = nt_tiles > 1 ? segk[28 + r] : -INFINITY, l1 = nt_tiles > 1 ? segk[32 + r] : 0.f;
-          const float M = fmaxf(m0, m1);
-          float* pr = a.part + (rec_idx * kRows + r) * kRecFloats;
-          pr[kD] = M;
-          pr[kD + 1] = l0 * ex2(m0 - M) + (nt_tiles > 1 ? l1 * ex2(m1 - M) : 0.f);
-        }
-        __threadfence();
         const int64_t vf = vof(part, sg.s * part.Ts), vl = vof(part, (sg.s + 1) * part.Ts - 1);
         const int nseg = static_cast<int>(vl - vf + 1);
         const int old = atomicAdd(A.counters + sg.s, 1);
@@ -1153,17 +1109,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
           reinterpret_cast<int64_t*>(red)[1] = vl;
         }
       }
-      named_sync(2, 384);
+      named_sync(2, 256);
       if (merge_s[1]) break;
       if (merge_s[0]) {
-        // All three groups: rows merged by the value group (thread =
-        // coordinate), then out = Pi_V^T o_rot with the input coordinates j
-        // split in three (thread = output coordinate), partial sums in smem.
+        // Records of the stream (two per segment), merged online by group 0
+        // (thread = coordinate, four records at a time with all loads in
+        // flight); then out = Pi_V^T o_rot with the input coordinates split in
+        // two (thread = output coordinate), partial sums through smem.
         const int64_t vf = reinterpret_cast<const int64_t*>(red)[0], vl = reinterpret_cast<const int64_t*>(red)[1];
-        const int crd = u & 127, part3 = u >> 7;
-        if (is_val) {
-          // The stream's records, four at a time with all loads in flight,
-          // merged online (running maximum, sum and rotated output per row).
+        const int crd = u & 127, half = u >> 7;
+        if (half == 0) {
           float M[kRows], L[kRows], O[kRows];
 #pragma unroll
           for (int r = 0; r < kRows; ++r) {
@@ -1171,17 +1126,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
             L[r] = 0.f;
             O[r] = 0.f;
           }
-          for (int64_t v0 = vf; v0 <= vl; v0 += 4) {
-            float mk[4][kRows], lk[4][kRows], ok[4][kRows];
+          const int64_t r0 = (vf + sg.s) * 2, r1 = (vl + sg.s) * 2 + 1;
+          for (int64_t c0 = r0; c0 <= r1; c0 += 4) {
+            float mk[4][kRows], lk[4][kRows], ok4[4][kRows];
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
               for (int r = 0; r < kRows; ++r) {
-                const bool has = v0 + kk <= vl;
-                const float* pr = a.part + ((v0 + kk + sg.s) * kRows + r) * kRecFloats;
+                const bool has = c0 + kk <= r1;
+                const float* pr = a.part + ((c0 + kk) * kRows + r) * kRecFloats;
                 mk[kk][r] = has ? __ldcg(pr + kD) : -INFINITY;
                 lk[kk][r] = has ? __ldcg(pr + kD + 1) : 0.f;
-                ok[kk][r] = has ? __ldcg(pr + crd) : 0.f;
+                ok4[kk][r] = has ? __ldcg(pr + crd) : 0.f;
               }
 #pragma unroll
             for (int r = 0; r < kRows; ++r) {
@@ -1195,7 +1151,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
               for (int kk = 0; kk < 4; ++kk) {
                 const float wgt = mk[kk][r] == -INFINITY ? 0.f : ex2(mk[kk][r] - Mn);
                 L[r] = fmaf(lk[kk][r], wgt, L[r]);
-                O[r] = fmaf(ok[kk][r], wgt, O[r]);
+                O[r] = fmaf(ok4[kk][r], wgt, O[r]);
               }
               M[r] = Mn;
             }
@@ -1203,33 +1159,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
 #pragma unroll
           for (int r = 0; r < kRows; ++r) qx[r * kD + crd] = L[r] > 0.f ? O[r] / L[r] : 0.f;
         }
-        named_sync(2, 384);
+        named_sync(2, 256);
         const float* PV = a.PiV + int64_t(kv) * a.pi_stride;
-        const int j_lo = part3 * 43, j_n = part3 == 2 ? 42 : 43;
+        const int j_lo = half * 64;
         float o4[kRows] = {0.f, 0.f, 0.f, 0.f};
-        {
-          float pv[43];
+#pragma unroll 1
+        for (int jb = 0; jb < 64; jb += 32) {
+          float pv[32];
 #pragma unroll
-          for (int k = 0; k < 43; ++k) pv[k] = k < j_n ? __ldg(PV + int64_t(j_lo + k) * kD + crd) : 0.f;
+          for (int kk = 0; kk < 32; ++kk) pv[kk] = __ldg(PV + int64_t(j_lo + jb + kk) * kD + crd);
 #pragma unroll
-          for (int k = 0; k < 43; ++k) {
-            const int jj = j_lo + (k < j_n ? k : 0);
+          for (int kk = 0; kk < 32; ++kk) {
 #pragma unroll
-            for (int r = 0; r < kRows; ++r) o4[r] = fmaf(pv[k], qx[r * kD + jj], o4[r]);
+            for (int r = 0; r < kRows; ++r) o4[r] = fmaf(pv[kk], qx[r * kD + j_lo + jb + kk], o4[r]);
           }
         }
-        // Parts 1 and 2 leave their sums in qr / sv; part 0 (the value group)
-        // adds them and stores the rows.
-        if (part3 > 0) {
-          float* dst = part3 == 1 ? qr : sv;
+        if (half == 1) {
 #pragma unroll
-          for (int r = 0; r < kRows; ++r) dst[r * kD + crd] = o4[r];
+          for (int r = 0; r < kRows; ++r) qr[r * kD + crd] = o4[r];
         }
-        named_sync(2, 384);
-        if (part3 == 0) {
+        named_sync(2, 256);
+        if (half == 0) {
 #pragma unroll
           for (int r = 0; r < kRows; ++r) {
-            const float v = o4[r] + qr[r * kD + crd] + sv[r * kD + crd];
+            const float v = o4[r] + qr[r * kD + crd];
             const int64_t oi = qrow(r) * kD + crd;
             if (a.out_dtype == 0) reinterpret_cast<float*>(a.out)[oi] = v;
             else reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(v);
@@ -1237,7 +1190,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
           if (crd == 0) A.counters[sg.s] = 0;    // ready for the next call
         }
       }
-      named_sync(2, 384);                         // qx is the next prologue's again
+      named_sync(2, 256);                         // qx / qr are the next prologue's again
     }
   }
 
@@ -1255,7 +1208,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
 struct FusedPlan {
   int64_t T, Ts, streams;
   int V;
-  size_t off_part, bytes;
+  size_t off_qprep, off_part, bytes;
 };
 // Partition and workspace of a call on `grid` CTAs: [arrival counters, one per
 // stream | partial records, one per (virtual CTA, stream) pair index v + s].
@@ -1267,8 +1220,9 @@ FusedPlan fused_plan(const DecodeShape& s, int grid) {
   const int64_t vmin = (p.T + kMaxSegTiles - 1) / kMaxSegTiles;
   // Every physical CTA gets the same number of virtual ones.
   p.V = static_cast<int>(((std::max<int64_t>(vmin, 1) + grid - 1) / grid) * grid);
-  p.off_part = ((size_t(p.streams) * sizeof(int) + 255) / 256) * 256;
-  p.bytes = p.off_part + size_t(p.V + p.streams) * kRows * kRecFloats * sizeof(float);
+  p.off_qprep = ((size_t(p.streams) * sizeof(int) + 255) / 256) * 256;
+  p.off_part = p.off_qprep + size_t(p.streams) * kQPrepStride;
+  p.bytes = p.off_part + size_t(p.V + p.streams) * 2 * kRows * kRecFloats * sizeof(float);
   return p;
 }
 
@@ -1310,8 +1264,12 @@ cudaError_t tc_decode_launch(const DecodeArgs& v, void* workspace, cudaStream_t 
   A.Ts = p.Ts;
   A.V = p.V;
   A.counters = static_cast<int*>(workspace);
+  A.qprep = static_cast<unsigned char*>(workspace) + p.off_qprep;
   A.v.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.off_part);
   e = cudaMemsetAsync(A.counters, 0, size_t(p.streams) * sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  decode_qprep_kernel<<<static_cast<unsigned>(p.streams), 256, 0, st>>>(A);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   switch (v.sh.kbits) {
     case 2:
