@@ -59,7 +59,11 @@ typedef enum {
 #define TQ_DEV_BAD_CODEBOOK   0x1  /* boundaries not strictly increasing       */
 #define TQ_DEV_BAD_POSITION   0x2  /* a RoPE position was negative            */
 #define TQ_DEV_TIMEOUT        0x4  /* a kernel gave up waiting on its own pipeline
-                                      (bounded wait); outputs of that call are invalid */
+                                      (bounded wait); outputs of that call are invalid.
+                                      The pipeline waits of the tensor-core kernels
+                                      give up after 2 s, or after the number of ns in
+                                      the environment variable TQ_TEST_WAIT_NS (read
+                                      at each call; for tests of this path). */
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
 
@@ -322,6 +326,16 @@ const char* tq_last_error_string(void);
 
 /* Library version string. */
 const char* tq_version(void);
+
+/* ------------------------------------------------------------------------
+ * tq_kernel_launches — diagnostic, no counterpart in the pages.
+ *
+ * Number of kernels this library has launched (or recorded into a CUDA graph
+ * under stream capture) since it was loaded, summed over all host threads and
+ * devices. Library-internal memsets are not counted. Callers take the
+ * difference of two readings around a region.
+ * ---------------------------------------------------------------------- */
+uint64_t tq_kernel_launches(void);
 
 #ifdef __cplusplus
 }

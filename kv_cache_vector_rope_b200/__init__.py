@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_PKG, "libtq.so")
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(5)
 TQ_F32, TQ_BF16 = 0, 1
-TQ_DEV_BAD_CODEBOOK, TQ_DEV_BAD_POSITION = 0x1, 0x2
+TQ_DEV_BAD_CODEBOOK, TQ_DEV_BAD_POSITION, TQ_DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 _STATUS = {1: "TQ_ERR_INVALID_ARG", 2: "TQ_ERR_UNSUPPORTED", 3: "TQ_ERR_CUDA", 4: "TQ_ERR_WORKSPACE"}
 
@@ -72,6 +72,7 @@ _SIGNATURES = {
     "tq_rotate_normalize": (ctypes.c_int, [_I32, _P, _I64, _P, _P, ctypes.POINTER(_I64)]),
     "tq_last_error_string": (ctypes.c_char_p, []),
     "tq_version": (ctypes.c_char_p, []),
+    "tq_kernel_launches": (ctypes.c_uint64, []),
 }
 
 
@@ -311,3 +312,8 @@ def tq_last_error_string() -> str:
 
 def tq_version() -> str:
     return _lib.tq_version().decode()
+
+
+def tq_kernel_launches() -> int:
+    """Kernels the library has launched (or captured) since it was loaded."""
+    return int(_lib.tq_kernel_launches())

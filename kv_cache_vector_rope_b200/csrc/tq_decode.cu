@@ -686,6 +686,7 @@ cudaError_t launch_rows(const DecodeArgs& a, cudaStream_t st) {
     if (COMBINE) decode_combine_rows<64><<<grid, 64, 0, st>>>(a);
     else decode_prologue_rows<64><<<grid, 64, 0, st>>>(a);
   }
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -704,6 +705,7 @@ cudaError_t launch_blk(const DecodeArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<static_cast<unsigned>(rb.n_blocks), kBlkThreads, smem, st>>>(a, rb);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -722,6 +724,7 @@ cudaError_t launch_v2(const DecodeArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   dim3 grid(a.sh.n_splits, static_cast<unsigned>(int64_t(a.sh.batch) * a.sh.hkv * a.sh.row_blocks));
   decode_main_v2<D, R, KB><<<grid, kT2, Sm::kBytes, st>>>(a);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -751,6 +754,7 @@ cudaError_t launch_main(const DecodeArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   dim3 grid(a.sh.n_splits, static_cast<unsigned>(int64_t(a.sh.batch) * a.sh.hkv * a.sh.row_blocks));
   decode_main<D, R><<<grid, kT, smem, st>>>(a);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -37,15 +37,21 @@
 //               and restarted in the other TMEM region.
 //   Combine     the last segment of a stream to finish (a per-stream arrival
 //               counter) merges the stream's records and applies Pi_V^T.
-// Roles (512 threads, one CTA per SM):
-//   warp 0       bulk copies of the index and sign planes into a 4-stage ring
-//   warp 1       TMEM owner and score MMA issuer   (warp-uniform loop, elected lane)
-//   warp 2       PV MMA issuer
-//   warps 4-7    key operands into TMEM            (thread = token)
-//   warps 8-11   value operands into smem, folds, combine (thread = token / coordinate)
-//   warps 12-15  scores, softmax, weights          (thread = token)
-// Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT and the CTA
-// drains its copies and MMAs before it frees TMEM and returns.
+// Roles (640 threads, one CTA per SM):
+//   warp 0        bulk copies: the index and sign planes into a 4-stage ring,
+//                 each segment's query side into one of two copies
+//   warp 1        TMEM owner and score MMA issuer   (warp-uniform loop, elected lane)
+//   warp 2        PV MMA issuer
+//   warp 3        the codebook limb tables (prologue only)
+//   warps 4-11    two key groups, alternate tiles: key operands into TMEM and
+//                 value operands into smem        (thread = token)
+//   warps 12-19   two softmax groups, alternate tiles of a segment: scores,
+//                 softmax, weights, folds; together the arrival and the combine
+//                 (thread = token / coordinate)
+// Every wait is bounded (2 s; the pipeline waits take the launch's limit, which
+// the environment variable TQ_TEST_WAIT_NS can shorten); a timeout sets
+// TQ_DEV_TIMEOUT and the CTA drains its copies and MMAs (full 2 s limit)
+// before it frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -124,6 +130,7 @@ struct FusedArgs {
   int V;               // virtual CTAs
   int* counters;       // [streams] arrivals (zero at launch)
   unsigned char* qprep;  // [streams][kQPrepStride] query side of the score MMAs
+  uint64_t wait_ns;    // pipeline wait limit (drains keep 2 s)
 };
 
 // int8 limbs of the key codebook (three) and the value codebook (two),
@@ -477,11 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
   const DecodeShape& sh = a.sh;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Sm::kOffBar);
   uint64_t* st_full = bars;                       // [kStages] loader (tx)
-  uint64_t* st_empty = bars + kStages;            // [kStages] the tile's key group + value/softmax group
+  uint64_t* st_empty = bars + kStages;            // [kStages] the tile's key group read the stage
   uint64_t* a_full = bars + 2 * kStages;          // [2] key group of the buffer
   uint64_t* s_full = a_full + 2;                  // [2] score commit (also frees the A operand)
   uint64_t* ds_free = s_full + 2;                 // [2] the group read the score columns
-  uint64_t* pv_ready = ds_free + 2;               // [kNVh] the group wrote the value operand and P
+  uint64_t* pv_ready = ds_free + 2;               // [kNVh] value operand (key group) and P (softmax group) written
   uint64_t* pv_full = pv_ready + kNVh;            // [kNVh] PV commit (frees the value operand and P)
   uint64_t* bt_full = pv_full + kNVh;             // [2] per segment parity: the query-side copy (tx)
   uint64_t* bt_free = bt_full + 2;                // [2] score issuer: the segment's score MMAs are done
@@ -508,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 8);
+      mbar_init(&st_empty[s], 4);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&a_full[b], 4);
@@ -520,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       mbar_init(&drain[b], 1);
     }
     for (int x = 0; x < kNVh; ++x) {
-      mbar_init(&pv_ready[x], 4);
+      mbar_init(&pv_ready[x], 8);
       mbar_init(&pv_full[x], 1);
     }
     for (int x = 0; x < 4; ++x) {
@@ -552,6 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
     // ------------------------------------------------------------- loader
     if (lane == 0) {
       int j = 0;
+      int bt_last[2] = {0, 0};                   // 1 + index of the last segment copied into each copy
       bool ok = true;
       SegIter it(part);
       Seg sg;
@@ -561,13 +569,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
           // The segment's query side (B tiles and row constants) into copy ib,
           // once the score MMAs of segment idx - 2 are done with it.
           const int ib = sg.idx & 1;
-          if (*abort_s || !mbar_wait(&bt_free[ib], ((sg.idx >> 1) & 1) ^ 1)) { ok = false; break; }
+          if (*abort_s || !mbar_wait(&bt_free[ib], ((sg.idx >> 1) & 1) ^ 1, A.wait_ns)) { ok = false; break; }
           mbar_expect_tx(&bt_full[ib], kQPrepBytes);
           bulk_g2s(sm + Sm::kOffB + ib * kBStride, A.qprep + sg.s * kQPrepStride, kQPrepBytes, &bt_full[ib]);
+          bt_last[ib] = sg.idx + 1;
         }
         for (int64_t tt = sg.t0; tt < sg.t1; ++tt, ++j) {
           const int s = j % kStages;
-          if (*abort_s || !mbar_wait(&st_empty[s], ((j / kStages) & 1) ^ 1)) { ok = false; break; }
+          if (*abort_s || !mbar_wait(&st_empty[s], ((j / kStages) & 1) ^ 1, A.wait_ns)) { ok = false; break; }
           const int64_t t0 = tt * kTT;
           const int nt = static_cast<int>((sh.n_ctx - t0 < kTT ? sh.n_ctx - t0 : int64_t(kTT)));
           const uint32_t bk = nt * kRbk, bs = nt * 16, bv = nt * 48;
@@ -579,11 +588,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
         }
       }
       if (!ok && !*abort_s) fail();
-      // Drain: the last copy into every stage has landed before the CTA exits.
+      // Drain: the last copy into every stage and into both query-side
+      // copies has landed before the CTA exits.
       for (int k = 1; k <= kStages && j - k >= 0; ++k) {
         const int jj = j - k;
         mbar_wait(&st_full[jj % kStages], (jj / kStages) & 1);
       }
+      for (int ib = 0; ib < 2; ++ib)
+        if (bt_last[ib] > 0) mbar_wait(&bt_full[ib], ((bt_last[ib] - 1) >> 1) & 1);
     }
   } else if (warp == kWScore || warp == kWPv) {
     // ------------------------------------------ MMA issuers (one warp each)
@@ -607,13 +619,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       const int ib = sg.idx & 1;
       const int nt_tiles = static_cast<int>(sg.t1 - sg.t0);
       if (warp == kWScore &&
-          !__all_sync(0xffffffffu, mbar_wait(&bt_full[ib], (sg.idx >> 1) & 1))) { ok = false; break; }
+          !__all_sync(0xffffffffu, mbar_wait(&bt_full[ib], (sg.idx >> 1) & 1, A.wait_ns))) { ok = false; break; }
       for (int tj = 0; tj < nt_tiles; ++tj, ++j) {
         const int b = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         if (__any_sync(0xffffffffu, *abort_s != 0)) { ok = false; break; }
         if (warp == kWScore) {
-          const bool w = mbar_wait(&a_full[b], ph) && mbar_wait(&ds_free[b], ph ^ 1);
+          const bool w = mbar_wait(&a_full[b], ph, A.wait_ns) && mbar_wait(&ds_free[b], ph ^ 1, A.wait_ns);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + kColDs + b * 32;
@@ -634,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
           }
         } else {
           const int xb = j % kNVh;                  // value operand / P buffer of the tile
-          const bool w = mbar_wait(&pv_ready[xb], (j / kNVh) & 1);
+          const bool w = mbar_wait(&pv_ready[xb], (j / kNVh) & 1, A.wait_ns);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           tc_fence_after();
           const bool flip = recs[(j & 7) * 16 + 1] != 0u;
@@ -652,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
           const int X = 2 * g + static_cast<int>((pcur >> g) & 1u);
           const uint32_t nclose = (pcl >> (8 * X)) & 0xFFu;
           if (fresh && nclose > 0 &&
-              !__all_sync(0xffffffffu, mbar_wait(&reg_free[X], (nclose - 1) & 1))) { ok = false; break; }
+              !__all_sync(0xffffffffu, mbar_wait(&reg_free[X], (nclose - 1) & 1, A.wait_ns))) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + kColDo + X * 32;
           const uint64_t pb = p_desc0 + ((xb * 2048) >> 4);
@@ -684,7 +696,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
   } else if (warp >= kWKey0 && warp < kWVs0) {
     // ---------------------------------- key operands (TMEM), two groups of 4 warps
     // Key group kg builds the A operand of the tiles with j % 2 == kg (its
-    // own TMEM buffer).
+    // own TMEM buffer), then their value operand (smem buffer j % 3); it is
+    // the only reader of the stage.
     const int kg = (warp - kWKey0) >> 2;
     const int q = warp & 3;                       // lane quadrant
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -696,6 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       k2[u] = tab[4 + u];
       k3[u] = tab[8 + u];
     }
+    const uint32_t v1t[2] = {tab[12], tab[13]}, v2t[2] = {tab[16], tab[17]};
     int j = 0;
     bool stop = false;
     SegIter it(part);
@@ -706,26 +720,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
         const int s = j % kStages;
         const int b = j & 1;
         if (b != kg) continue;
-        if (!__all_sync(0xffffffffu, mbar_wait(&st_full[s], (j / kStages) & 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&st_full[s], (j / kStages) & 1, A.wait_ns))) {
           if (lane == 0) fail();
           stop = true;
           break;
         }
-        const unsigned char* st = sm + s * Sm::kStageStride;
         // The row's code words stay in shared memory until the limbs are
-        // built (read KB words per 32 coordinates); the stage is released
-        // after the last read.
+        // built (read KB words per 32 coordinates, value codes 3 words per 32);
+        // the stage is released after the last read. (Loops are not unrolled:
+        // the kernel's five roles share the instruction cache.)
+        const unsigned char* st = sm + s * Sm::kStageStride;
         const uint32_t* wrow = reinterpret_cast<const uint32_t*>(st + row * kRbk);
         const uint4 sg4 = reinterpret_cast<const uint4*>(st + Sm::kOffKs + row * 16)[0];
-        if (!__all_sync(0xffffffffu, mbar_wait(&a_free[b], ((j >> 1) & 1) ^ 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&a_free[b], ((j >> 1) & 1) ^ 1, A.wait_ns))) {
           if (lane == 0) fail();
           stop = true;
           break;
         }
         tc_fence_after();
         const uint32_t acol = lane_addr + kColA + b * 128;
-        // 32 coordinates per iteration (KB words of codes): nibble selectors,
-        // then the three limbs of each coordinate by byte permutes into 8 TMEM
+        // 32 coordinates per step (KB words of codes): nibble selectors, then
+        // the three limbs of each coordinate by byte permutes into 8 TMEM
         // columns per limb.
 #pragma unroll 1
         for (int qq = 0; qq < 4; ++qq) {
@@ -760,28 +775,70 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
             tmem_st8(acol + limb * 32 + qq * 8, v8);
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&st_empty[s]);
-        uint32_t v[32];
-        // Sign chunk: column 4 m + u = sign word u AND (0x01010101 << m).
-        const uint32_t swd[4] = {sg4.x, sg4.y, sg4.z, sg4.w};
+        {
+          uint32_t v[32];
+          // Sign chunk: column 4 m + u = sign word u AND (0x01010101 << m).
+          const uint32_t swd[4] = {sg4.x, sg4.y, sg4.z, sg4.w};
 #pragma unroll
-        for (int m = 0; m < 8; ++m)
+          for (int m = 0; m < 8; ++m)
 #pragma unroll
-          for (int u = 0; u < 4; ++u) v[4 * m + u] = swd[u] & (0x01010101u << m);
-        tmem_st32(acol + 96, v);
+            for (int u = 0; u < 4; ++u) v[4 * m + u] = swd[u] & (0x01010101u << m);
+          tmem_st32(acol + 96, v);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[b]);
+        // -- value operand of the tile (thread = token): two int8 limbs of the
+        // value codebook, one 128-byte M-major row per token and limb, into
+        // buffer xb = j % 3 once the product of tile j - 3 has read it.
+        const int xb = j % kNVh;
+        if (!__all_sync(0xffffffffu, mbar_wait(&vh_free[xb], ((j / kNVh) & 1) ^ 1, A.wait_ns))) {
+          if (lane == 0) fail();
+          stop = true;
+          break;
+        }
+        {
+          const uint32_t* vrow = reinterpret_cast<const uint32_t*>(st + Sm::kOffVi + row * 48);
+          unsigned char* vh = sm + Sm::kOffVh + xb * Sm::kVhBytes;
+          const int atom = row >> 3, r8 = row & 7;
+#pragma unroll 1
+          for (int c2 = 0; c2 < 4; ++c2) {
+            const uint32_t x4[4] = {vrow[3 * c2], vrow[3 * c2 + 1], vrow[3 * c2 + 2], 0u};
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {          // 16 coordinates = 6 bytes of codes
+              uint32_t o1[4], o2[4];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {           // 8 codes per half
+                const int g = 2 * cc + h;
+                const int off = 3 * g, wi = off >> 2, shf = 8 * (off & 3);
+                const uint32_t x = shf == 0 ? x4[wi] : __funnelshift_r(x4[wi], x4[wi + 1], shf);
+                const uint32_t nb = nibbles3(x);
+                o1[2 * h] = prmt(v1t[0], v1t[1], nb);
+                o1[2 * h + 1] = prmt(v1t[0], v1t[1], nb >> 16);
+                o2[2 * h] = prmt(v2t[0], v2t[1], nb);
+                o2[2 * h + 1] = prmt(v2t[0], v2t[1], nb >> 16);
+              }
+              const int c16 = 2 * c2 + cc;
+              const uint32_t off = atom * 1024 + r8 * 128 + ((c16 ^ r8) << 4);
+              *reinterpret_cast<uint4*>(vh + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+              *reinterpret_cast<uint4*>(vh + kTT * 128 + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&st_empty[s]);
+          mbar_arrive(&pv_ready[xb]);
+        }
       }
     }
   } else if (warp >= kWVs0) {
-    // ---------------------------------------- value + softmax groups (2 x 4 warps)
-    // Group g takes the segment's tiles tj with tj % 2 == g: it builds the
-    // tile's value operand, turns its scores into weights and folds its own
-    // TMEM regions (2g, 2g + 1). Both groups share the segment prologue, the
-    // arrival and the combine (256 threads on barrier 2).
+    // ---------------------------------------------- softmax groups (2 x 4 warps)
+    // Group g takes the segment's tiles tj with tj % 2 == g: it turns their
+    // scores into weights and folds its own TMEM regions (2g, 2g + 1). Both
+    // groups share the arrival and the combine (256 threads on barrier 2).
     const int grp = (warp - kWVs0) >> 2;          // 0 or 1
     const int gbar = grp == 0 ? 1 : 4;            // the group's named barrier (128 threads)
     const int u = tid - kWVs0 * 32;               // 0..255
@@ -790,7 +847,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const float alpha = static_cast<float>(dev::kSqrtHalfPi / kD);
     constexpr float kLog2e = 1.4426950408889634f;
-    const uint32_t v1t[2] = {tab[12], tab[13]}, v2t[2] = {tab[16], tab[17]};
     int j = 0;                                    // CTA-local tile counter
     bool stop = false;
     uint32_t gcur = 0u;                           // region in use: 2 grp + gcur
@@ -827,7 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       norm_fetch(1);
       norm_fetch(2);
       // ---------------- the segment's query side (copied in by the loader)
-      if (!__all_sync(0xffffffffu, mbar_wait(&bt_full[ib], (sg.idx >> 1) & 1)) && lane == 0) fail();
+      if (!__all_sync(0xffffffffu, mbar_wait(&bt_full[ib], (sg.idx >> 1) & 1, A.wait_ns)) && lane == 0) fail();
       const float* qc = reinterpret_cast<const float*>(sm + Sm::kOffB + ib * kBStride + 4 * 2048);
       // ---------------- the group's tiles
       float kq[kRows], ks2[kRows], ssum[kRows];
@@ -853,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       auto fold = [&](const float (&m_seg)[kRows]) -> bool {
         const int X = 2 * grp + static_cast<int>(gcur);
         const uint32_t nclose = (gcl >> (8 * gcur)) & 0xFFu;
-        if (!__all_sync(0xffffffffu, mbar_wait(&reg_done[X], nclose & 1))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&reg_done[X], nclose & 1, A.wait_ns))) return false;
         tc_fence_after();
         uint32_t dv[32];
         tmem_ld32(lane_addr + kColDo + X * 32, dv);
@@ -881,7 +937,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
       for (int k = 0; 2 * k + grp < nt_tiles; ++k) {
         const int tj = 2 * k + grp;
         const int jt = j0 + tj;
-        const int b = jt & 1, s = jt % kStages;
+        const int b = jt & 1;
         const int64_t t0 = (sg.t0 + tj) * kTT;
         const int nt = static_cast<int>((sh.n_ctx - t0 < kTT ? sh.n_ctx - t0 : int64_t(kTT)));
         const bool valid = lrow < nt;
@@ -890,7 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
         cp_async_wait<3>();
         const float* slot = nring + (k & 3) * (3 * kTT);
         const float kn = slot[lrow], rn = slot[kTT + lrow], vn = slot[2 * kTT + lrow];
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (jt >> 1) & 1));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (jt >> 1) & 1, A.wait_ns));
         tc_fence_after();
         // MSE part: weights 1, 1/128, 1/128^2 of the key-limb products
         // (weight 3 is below 1e-6 of the first); sign part: four limbs.
@@ -1004,43 +1060,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(FusedArgs A) 
           l_part[r] += p[r];
           X[r] = valid ? __float2uint_rn(x[r] * 16777216.f) : 0u;
         }
-        // -- value operand of the tile (thread = token): two int8 limbs of the
-        // value codebook, one 128-byte M-major row per token and limb.
-        // (Built after the scores: the buffer, xb = jt % 3, is freed by the
-        // product of tile jt - 3, which is usually done by now.)
+        // -- weights of the tile into P[xb] (xb = jt % 3), once the product
+        // of tile jt - 3 has read it; the key group builds the value operand.
         const int xb = jt % kNVh;
-        const bool okv = mbar_wait(&st_full[s], (jt / kStages) & 1) && mbar_wait(&vh_free[xb], ((jt / kNVh) & 1) ^ 1);
-        if (!__all_sync(0xffffffffu, okv) && lane == 0) fail();
-        {
-          const uint32_t* wrow = reinterpret_cast<const uint32_t*>(sm + s * Sm::kStageStride + Sm::kOffVi + lrow * 48);
-          unsigned char* vh = sm + Sm::kOffVh + xb * Sm::kVhBytes;
-          const int atom = lrow >> 3, r8 = lrow & 7;
-#pragma unroll 1
-          for (int c2 = 0; c2 < 4; ++c2) {
-            const uint32_t x4[4] = {wrow[3 * c2], wrow[3 * c2 + 1], wrow[3 * c2 + 2], 0u};
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {          // 16 coordinates = 6 bytes of codes
-              uint32_t o1[4], o2[4];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {           // 8 codes per half
-                const int g = 2 * cc + h;
-                const int off = 3 * g, wi = off >> 2, shf = 8 * (off & 3);
-                const uint32_t x = shf == 0 ? x4[wi] : __funnelshift_r(x4[wi], x4[wi + 1], shf);
-                const uint32_t nb = nibbles3(x);
-                o1[2 * h] = prmt(v1t[0], v1t[1], nb);
-                o1[2 * h + 1] = prmt(v1t[0], v1t[1], nb >> 16);
-                o2[2 * h] = prmt(v2t[0], v2t[1], nb);
-                o2[2 * h + 1] = prmt(v2t[0], v2t[1], nb >> 16);
-              }
-              const int c16 = 2 * c2 + cc;
-              const uint32_t off = atom * 1024 + r8 * 128 + ((c16 ^ r8) << 4);
-              *reinterpret_cast<uint4*>(vh + off) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-              *reinterpret_cast<uint4*>(vh + kTT * 128 + off) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&st_empty[s]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&vh_free[xb], ((jt / kNVh) & 1) ^ 1, A.wait_ns)) && lane == 0) fail();
         *reinterpret_cast<uint4*>(sm + Sm::kOffP + xb * 2048 + lrow * 16) = make_uint4(X[0], X[1], X[2], X[3]);
         if (lrow == 0) recs[(jt & 7) * 16 + 1] = flip ? 1u : 0u;
         fence_proxy_async_smem();
@@ -1264,11 +1287,13 @@ cudaError_t tc_decode_launch(const DecodeArgs& v, void* workspace, cudaStream_t 
   A.Ts = p.Ts;
   A.V = p.V;
   A.counters = static_cast<int*>(workspace);
+  A.wait_ns = pipeline_wait_ns();
   A.qprep = static_cast<unsigned char*>(workspace) + p.off_qprep;
   A.v.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + p.off_part);
   e = cudaMemsetAsync(A.counters, 0, size_t(p.streams) * sizeof(int), st);
   if (e != cudaSuccess) return e;
   decode_qprep_kernel<<<static_cast<unsigned>(p.streams), 256, 0, st>>>(A);
+  count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   switch (v.sh.kbits) {
@@ -1286,6 +1311,7 @@ cudaError_t tc_decode_launch(const DecodeArgs& v, void* workspace, cudaStream_t 
       break;
   }
   if (e != cudaSuccess) return e;
+  count_launch();
   return cudaGetLastError();
 }
 

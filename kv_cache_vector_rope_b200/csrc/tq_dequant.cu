@@ -105,6 +105,7 @@ extern "C" tq_status tq_dequantize(const tq_layout* layout, int32_t is_key, int6
                 planes->sign, planes->norm, planes->rnorm, Pi, vectors_per_pi, pi_stride, S, centroids, out,
                 out_dtype == TQ_F32 ? 0 : 1, out_stride};
   dequant_kernel<<<static_cast<unsigned>(n_vectors), 128, 2 * d * sizeof(float), static_cast<cudaStream_t>(stream)>>>(a);
+  count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_dequantize launch: %s", cudaGetErrorString(e));
   return TQ_OK;

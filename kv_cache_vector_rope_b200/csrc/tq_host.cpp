@@ -8,8 +8,10 @@
 // computed once. gist.science TurboESM section 2C — separate K / V tables
 // fitted to their own rotated coordinates (empirical mode).
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -234,9 +236,26 @@ tq_status lloyd_empirical(const float* samples, int64_t ns, int bits, std::vecto
 }
 
 }  // namespace
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+uint64_t pipeline_wait_ns() {
+  const char* e = std::getenv("TQ_TEST_WAIT_NS");
+  if (e == nullptr || *e == 0) return 2000000000ull;
+  char* end = nullptr;
+  const unsigned long long v = std::strtoull(e, &end, 10);
+  return (end != e && v <= 2000000000ull) ? static_cast<uint64_t>(v) : 2000000000ull;
+}
+
 }  // namespace tq
 
 extern "C" {
+
+uint64_t tq_kernel_launches(void) { return tq::g_launches.load(std::memory_order_relaxed); }
 
 const char* tq_last_error_string(void) { return tq::g_last_error.c_str(); }
 

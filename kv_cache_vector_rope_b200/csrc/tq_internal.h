@@ -24,4 +24,12 @@ tq_status check_bits(int bits, const char* what);
 
 constexpr int kMaxD = 256;
 
+// Counts kernel launches issued by the library (tq_kernel_launches).
+void count_launch(int n = 1);
+
+// Limit of the tcgen05 kernels' pipeline waits, in ns: 2 s, or the value of
+// the environment variable TQ_TEST_WAIT_NS (tests shorten it to make the waits
+// run out). The waits that drain copies and MMAs before exit keep 2 s.
+uint64_t pipeline_wait_ns();
+
 }  // namespace tq

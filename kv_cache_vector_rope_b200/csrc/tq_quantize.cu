@@ -366,6 +366,7 @@ cudaError_t launch(const QuantArgs& a, cudaStream_t st) {
   const int64_t tiles = (a.n + kTV - 1) / kTV;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, int64_t(sms) * std::max(1, per_sm))));
   quantize_kernel<D><<<grid, kThreads, smem, st>>>(a);
+  count_launch();
   return cudaGetLastError();
 }
 

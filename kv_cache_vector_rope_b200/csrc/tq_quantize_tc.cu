@@ -34,8 +34,10 @@
 // launch, quantize_fixup, recomputes every flagged row exactly in fp64 (four
 // rows per warp: ||x||, y = Pi x, codes, r, p = S r) and overwrites it.
 //
-// Every wait is bounded (2 s); a timeout sets TQ_DEV_TIMEOUT in *d_status and
-// the CTA drains its own copies and MMAs, frees TMEM and returns.
+// Every wait is bounded (2 s; the pipeline waits take the launch's limit, which
+// the environment variable TQ_TEST_WAIT_NS can shorten); a timeout sets
+// TQ_DEV_TIMEOUT in *d_status and the CTA drains its own copies and MMAs (full
+// 2 s limit), frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -110,6 +112,7 @@ struct TcArgs {
   float* norm;
   float* rnorm;
   int32_t* d_status;
+  uint64_t wait_ns;     // pipeline wait limit (drains keep 2 s)
 };
 
 // Splits v into bf16 terms hi + mid + lo that add up to v to ~2^-25.
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         const int st = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
         if (*abort_s) break;
-        if (!mbar_wait(&empty[st], ph ^ 1)) { fail(); break; }
+        if (!mbar_wait(&empty[st], ph ^ 1, a.wait_ns)) { fail(); break; }
         mbar_expect_tx(&full[st], C::kTileBytes);
         unsigned char* dst = x_s + st * C::kTileBytes;
 #pragma unroll
@@ -366,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           last = globaltimer_ns();
         } else {
           __nanosleep(32);              // nothing ready: leave the issue slots to the other warps
-          if (globaltimer_ns() - last > 2000000000ull) {
+          if (globaltimer_ns() - last > a.wait_ns) {
             fail();
             break;
           }
@@ -387,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       const uint32_t ph = (it >> 1) & 1;
       const int64_t v = t * C::kM + row;
       const bool valid = v < a.n;
-      if (!__all_sync(0xffffffffu, mbar_wait(&yfull[wg], ph))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&yfull[wg], ph, a.wait_ns))) {
         if (lane == 0) fail();
         break;
       }
@@ -501,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         if (valid) a.norm[v] = nrm;
         const float rn = sqrtf(rsq);
         const float sband = kSignGuard * rn * rscale;
-        if (!__all_sync(0xffffffffu, mbar_wait(&pfull[wg], ph))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&pfull[wg], ph, a.wait_ns))) {
           if (lane == 0) fail();
           break;
         }
@@ -815,6 +818,7 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& map, cudaStream_t st) 
   const int64_t tiles = (a.n + 127) / 128;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   quantize_tc_kernel<D, KEY, BITS><<<grid, kThreads, C::kSmemBytes, st>>>(map, a);
+  count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   constexpr size_t fix_smem = FixCfg<D, KEY>::kBytes;
@@ -825,6 +829,7 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& map, cudaStream_t st) 
   const int64_t fix_ctas = (a.n + kFixList - 1) / kFixList;
   quantize_fixup<D, KEY, BITS><<<static_cast<int>(fix_ctas < sms ? (fix_ctas < 1 ? 1 : fix_ctas) : sms), kFixThreads,
                                  fix_smem, st>>>(a);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -859,7 +864,7 @@ tq_status tc_quantize(int d, bool is_key, int bits, const void* x, int64_t n, in
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   TcArgs a{static_cast<const __nv_bfloat16*>(x), n, row_stride, Pi, S, cent, bnd, out->idx,
-           is_key ? out->sign : nullptr, out->norm, is_key ? out->rnorm : nullptr, d_status};
+           is_key ? out->sign : nullptr, out->norm, is_key ? out->rnorm : nullptr, d_status, pipeline_wait_ns()};
   cudaError_t e;
   if (d == 128)
     e = is_key ? launch_bits<128, true>(bits, a, map, st) : launch_bits<128, false>(bits, a, map, st);

@@ -309,6 +309,7 @@ extern "C" tq_status tq_search_topk(const tq_layout* layout, const void* q, tq_d
   a.top_s = top_scores;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   search_prologue<<<n_queries, 128, d * sizeof(double) + d * sizeof(float), s>>>(a);
+  count_launch();
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) {
     const int nc = 1 << a.bits;
@@ -319,14 +320,17 @@ extern "C" tq_status tq_search_topk(const tq_layout* layout, const void* q, tq_d
       case 64:
         cudaFuncSetAttribute(search_main<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         search_main<64><<<grid, kSThreads, smem, s>>>(a);
+        count_launch();
         break;
       case 128:
         cudaFuncSetAttribute(search_main<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         search_main<128><<<grid, kSThreads, smem, s>>>(a);
+        count_launch();
         break;
       case 200:
         cudaFuncSetAttribute(search_main<200>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         search_main<200><<<grid, kSThreads, smem, s>>>(a);
+        count_launch();
         break;
       default:
         return fail(TQ_ERR_UNSUPPORTED, "tq_search_topk: d=%d not built (64, 128, 200)", d);
@@ -335,6 +339,7 @@ extern "C" tq_status tq_search_topk(const tq_layout* layout, const void* q, tq_d
   }
   if (e == cudaSuccess) {
     search_merge<<<(n_queries + 3) / 4, 128, 0, s>>>(a);
+    count_launch();
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_search_topk launch: %s", cudaGetErrorString(e));

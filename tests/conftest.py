@@ -26,3 +26,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    # Worst ratios of the GPU results against the literal tolerances.
+    try:
+        from tests import parity
+    except Exception:  # pragma: no cover
+        return
+    L = parity.LITERAL
+    if L["checks"]:
+        terminalreporter.write_line(
+            "literal-bound ratios (worst over all checks): score err / (1e-4 |s|) where |s| >= typical scale "
+            f"{L['score_rel']:.3g}; over all scores {L['score_rel_all']:.3g}; max |out err| / 2e-3 {L['out_abs']:.3g}")

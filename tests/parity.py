@@ -88,12 +88,25 @@ def value_planes(h: dict, bits: int) -> oa.ValuePlanes:
     return oa.ValuePlanes(h["idx"], h["norm"], bits)
 
 
+# Worst ratios against the literal tolerances (score: 1e-4 * |s_ref| alone, over
+# the scores with |s_ref| >= the typical scale, where a relative bound means
+# something; output: 2e-3 max-abs without the bf16 rounding allowance).
+# Collected by every check and printed at the end of the session.
+LITERAL = {"score_rel": 0.0, "score_rel_all": 0.0, "out_abs": 0.0, "checks": 0}
+
+
 def check_scores(gpu_scores: np.ndarray, ref_scores: np.ndarray, q_norm: np.ndarray, k_norm: np.ndarray, d: int):
-    """Rule 13 on [nq, N] score matrices; returns the worst ratio to the bound."""
+    """The SCORE rule on [nq, N] score matrices; returns the worst ratio to the bound."""
     typical = q_norm[:, None] * k_norm[None, :].astype(np.float64) / d
     bound = SCORE_RTOL * np.maximum(np.abs(ref_scores), typical)
     err = np.abs(gpu_scores.astype(np.float64) - ref_scores)
     worst = float((err / np.maximum(bound, 1e-300)).max())
+    rel = err / np.maximum(SCORE_RTOL * np.abs(ref_scores), 1e-300)
+    big = np.abs(ref_scores) >= typical
+    if big.any():
+        LITERAL["score_rel"] = max(LITERAL["score_rel"], float(rel[big].max()))
+    LITERAL["score_rel_all"] = max(LITERAL["score_rel_all"], float(rel.max()))
+    LITERAL["checks"] += 1
     assert np.all(err <= bound), f"score error {err.max()} exceeds bound (worst ratio {worst})"
     return worst
 
@@ -108,6 +121,8 @@ def check_out(gpu_out: torch.Tensor, ref: np.ndarray) -> float:
         spacing = np.exp2(np.floor(np.log2(np.maximum(m, 1e-30))) - 7)
         tol = OUT_ATOL + 0.5 * spacing
     err = np.abs(g - ref)
+    LITERAL["out_abs"] = max(LITERAL["out_abs"], float(err.max()) / OUT_ATOL)
+    LITERAL["checks"] += 1
     assert np.all(err <= tol), f"output max abs error {err.max()}"
     return float(err.max())
 

@@ -49,3 +49,31 @@ def test_two_rank_barrier_max_and_replica_seeds(tmp_path):
         assert float(slowest) == 1.5 * world          # max over ranks, seen by every rank
         assert backend == "gloo"
     assert len({row[3] for row in rows}) == world       # independent caches per rank
+
+
+def _bench(args, env_extra=None, timeout=300):
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_PORT")}
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, capture_output=True, text=True,
+                          env=env, timeout=timeout, cwd=ROOT)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the gloo path; GPU runs use NCCL")
+def test_bench_gpus_2_spawns_two_ranks_and_reports_them():
+    import json
+    r = _bench(["--impl", "reference", "--gpus", "2", "--config", "1", "--steps", "1", "--warmup", "0",
+                "--cpu-budget", "0.2"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout                   # rank 0 alone prints
+    res = json.loads(lines[0])
+    assert res["n_gpus"] == 2 and res["impl"] == "reference"
+    assert res["config"]["config_id"] == 1 and res["value"] > 0
+
+
+def test_bench_rejects_gpus_that_differ_from_the_launcher():
+    r = _bench(["--impl", "reference", "--gpus", "1", "--config", "1", "--steps", "1", "--warmup", "0"],
+               env_extra={"WORLD_SIZE": "2", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode != 0
+    assert "WORLD_SIZE=2" in r.stderr

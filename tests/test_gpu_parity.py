@@ -284,19 +284,27 @@ def test_full_llama_layer_sampled():
     c, _ = book(d, 3)
     N = shape.n_ctx
     out = torch.empty((shape.batch, shape.hq, 1, d), dtype=torch.bfloat16, device="cuda")
+    scores = torch.empty((shape.batch, shape.hq, 1, N), dtype=torch.float32, device="cuda")
     ws = tq.decode_workspace(lay, shape.batch, shape.hq, shape.hkv, 1, N)
-    tq.tq_decode_attention(lay, Q, kp, vp, shape.hkv, N, dev(Pi), dev(Pi), dev(S), dev(c), dev(c), out, ws)
+    tq.tq_decode_attention(lay, Q, kp, vp, shape.hkv, N, dev(Pi), dev(Pi), dev(S), dev(c), dev(c), out, ws,
+                           scores_out=scores)
     torch.cuda.synchronize()
     G = shape.hq // shape.hkv
     Qn = Q.float().cpu().numpy().astype(np.float64)
-    for (bi, kv) in [(0, 0), (3, 5), (7, 7)]:
-        rows = slice((bi * shape.hkv + kv) * N, (bi * shape.hkv + kv + 1) * N)
-        hk = {"idx": kp.idx[rows].cpu().numpy(), "sign": kp.sign[rows].cpu().numpy().view(np.uint32),
-              "norm": kp.norm[rows].cpu().numpy(), "rnorm": kp.rnorm[rows].cpu().numpy()}
-        hv = {"idx": vp.idx[rows].cpu().numpy(), "norm": vp.norm[rows].cpu().numpy()}
-        ref = oa.attention(Qn[bi, kv * G:(kv + 1) * G, 0], P.key_planes(hk, 3), P.value_planes(hv, 3),
-                           Pi, Pi, S, c, c)
-        P.check_out(out[bi, kv * G:(kv + 1) * G, 0], ref.out)
+    hk_all, hv_all = P.host_planes(kp), P.host_planes(vp)
+    sc_all = scores.cpu().numpy()
+    worst_s, worst_o = 0.0, 0.0
+    for bi in range(shape.batch):                      # every (batch, kv head) stream
+        for kv in range(shape.hkv):
+            rows = slice((bi * shape.hkv + kv) * N, (bi * shape.hkv + kv + 1) * N)
+            hk = {k: v[rows] for k, v in hk_all.items()}
+            hv = {k: v[rows] for k, v in hv_all.items()}
+            qs = Qn[bi, kv * G:(kv + 1) * G, 0]
+            ref = oa.attention(qs, P.key_planes(hk, 3), P.value_planes(hv, 3), Pi, Pi, S, c, c)
+            worst_s = max(worst_s, P.check_scores(sc_all[bi, kv * G:(kv + 1) * G, 0], ref.scores,
+                                                  np.linalg.norm(qs, axis=1), hk["norm"], d))
+            worst_o = max(worst_o, P.check_out(out[bi, kv * G:(kv + 1) * G, 0], ref.out))
+    print(f"full layer, 64 streams: worst score error / bound {worst_s:.3g}, worst |out - ref| {worst_o:.3g}")
 
 
 # ---------------------------------------------------------------------------
