@@ -86,7 +86,19 @@ WORKLOADS = {
 # (one kernel, one launch, ncu), divided by the units that launch processed.
 # An entry counts only while the listed sources still hash to `sha`; after any
 # change to them the traffic is reported as null until it is captured again.
-TRAFFIC = {}
+# Captured on the Llama-shaped cache at context 8192 (1 layer, 524,288 vectors
+# per call); at that size part of a call's output is still in L2 when the
+# kernel ends, so the write bytes are a lower bound. The quantise entries sum
+# the main kernel and its fixup (the call the roofline times).
+TRAFFIC = {
+    "decode_fused3_d128": {"bytes_per_unit": (65_943_552 + 246_272) / 524_288, "sha": "d958b2d61582ac83",
+                           "sources": ["tq_decode_tc.cu", "tq_decode_tc.h", "tq_sm100.cuh"]},
+    "quantize_tc_key3_d128": {"bytes_per_unit": (134_565_376 + 13_969_152 + 2_681_088) / 524_288,
+                              "sha": "3cf723122ba79b6b", "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
+    "quantize_tc_value3_d128": {"bytes_per_unit": (134_330_880 + 9_040_640 + 2_406_656) / 524_288,
+                                "sha": "3cf723122ba79b6b",
+                                "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
+}
 
 CSRC = os.path.join(ROOT, "kv_cache_vector_rope_b200", "csrc")
 
@@ -102,13 +114,15 @@ def parse(argv=None):
     p.add_argument("--context", type=int, default=32768,
                    help="config 3: context length (32768 = the full workload; smaller only for profiling)")
     p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--incremental-steps", type=int, default=8,
+                   help="config 3: generated tokens timed for the append-then-decode line (0: skip)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--cpu-budget", type=float, default=12.0,
                    help="seconds of oracle work for each of the two cpu_baseline timings")
     a = p.parse_args(argv)
     if a.steps is None:
-        a.steps = {1: 200, 2: 10, 3: 20, 4: 20, 5: 5}[a.config]
+        a.steps = {1: 5000, 2: 20, 3: 20, 4: 300, 5: 5}[a.config]
     return a
 
 
@@ -127,10 +141,13 @@ class ClockSampler:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
             self.proc = subprocess.Popen(["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            t0 = time.time()                      # the first sample precedes the timed region
+            while not self.lines and time.time() - t0 < 5.0:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
 
@@ -583,7 +600,25 @@ def run_c1(args, world, rank, tq):
     res["roofline"] = hbm_roofline("whole step (quantize_kernel x2 + decode kernels)", alg, ms * 1e-3, peaks,
                                    "fp32 K and V in (256 B each) + packed out (36 B key, 28 B value) per token")
     res["roofline"]["note"] = "latency-bound: the step moves ~0.2 MB; the fraction is not a target here"
-    return res, None
+    e2e = None
+    if not args.no_e2e:
+        hK, hV, hQ = (t.cpu().pin_memory() for t in (K, V, Q))
+        hout = torch.empty_like(out, device="cpu").pin_memory()
+
+        def e2e_step():
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            Q.copy_(hQ, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+
+        saved = args.e2e_steps
+        args.e2e_steps = max(saved, 200)
+        e2e = run_e2e_loop(args, world, e2e_step, n, "tokens/s", h2d=4 * (K.numel() + V.numel() + Q.numel()),
+                           d2h=4 * out.numel())
+        args.e2e_steps = saved
+        e2e["note"] = "per step: fp32 K, V and queries copied in, attention outputs read back"
+    return res, e2e
 
 
 # ---------------------------------------------------------------------------
@@ -673,9 +708,11 @@ def run_c2(args, world, rank, tq):
     att = alu_roofline("tq_decode_attention (1024 queries per head): decode_prologue + decode_main_v2<64> + "
                        "decode_combine, per layer", pairs * ops_pair, at_ms * 1e-3, T.clk,
                        f"{ops_pair} FP32 lane ops per (query, key) pair at d={d}; {pairs:,} pairs per step")
-    quant = hbm_roofline("tq_quantize_kv(keys, per-head Pi): quantize_kernel<64>", n * kb, kq_ms * 1e-3, peaks,
+    quant = hbm_roofline("tq_quantize_kv(keys, per-head Pi): quantize_tc_kernel<64,key,3,per-head> + quantize_fixup",
+                         n * kb, kq_ms * 1e-3, peaks,
                          f"bf16 in {2 * d} B + packed out {packed_bytes(d, 3, True)} B per key vector; {n:,} per call")
-    quant_v = hbm_roofline("tq_quantize_kv(values, per-head Pi): quantize_kernel<64>", n * vb, vq_ms * 1e-3, peaks,
+    quant_v = hbm_roofline("tq_quantize_kv(values, per-head Pi): quantize_tc_kernel<64,value,3,per-head> + "
+                           "quantize_fixup", n * vb, vq_ms * 1e-3, peaks,
                            f"bf16 in {2 * d} B + packed out {packed_bytes(d, 3, False)} B per value vector")
     if at_ms >= kq_ms + vq_ms:
         res["roofline"], res["roofline_quantize"], res["roofline_quantize_value"] = att, quant, quant_v
@@ -794,10 +831,56 @@ def run_c3(args, world, rank, tq):
                                           n_vec * dec_unit, dl_ms * 1e-3, peaks,
                                           f"{dec_unit} B per (token, kv head); {n_vec:,} per call",
                                           "decode_fused3_d128", n_vec)
+    if args.incremental_steps > 0:
+        res["incremental"] = run_incremental_c3(args, tq, lay, Q, kp, vp, out, ws, Pi, S, cd, td, status, shape,
+                                                world, L, dev)
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e_c3(args, tq, lay, K, V, Q, kp, vp, out, ws, Pi, S, cd, td, status, shape, world)
     return res, e2e
+
+
+def run_incremental_c3(args, tq, lay, Q, kp, vp, out, ws, Pi, S, cd, td, status, shape, world, L, dev):
+    """One generated token per step: every layer appends one key (RoPE at its position) and one value per
+    (batch, kv head) stream with tq_append_kv, then decodes over the grown cache. The cache holds N - T tokens
+    before the first of T steps (its capacity, ctx_stride, stays N)."""
+    B, HKV, D, N = shape.batch, shape.hkv, shape.d, shape.n_ctx
+    T = args.incremental_steps
+    streams = B * HKV
+    base = 500000.0                                # Llama-3.1 RoPE base
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    kn = torch.randn((T, L, streams, D), generator=g, device=dev).to(torch.bfloat16)
+    vn = torch.randn((T, L, streams, D), generator=g, device=dev).to(torch.bfloat16)
+    slots = [N - T + i for i in range(T)]
+    kpos = [torch.full((streams,), sl, dtype=torch.int32, device=dev) for sl in slots]
+    qpos = [torch.full((B, 1), sl, dtype=torch.int32, device=dev) for sl in slots]
+    marks = [(ev(), ev(), ev()) for _ in range(T)]
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = tq.tq_kernel_launches()
+    for i, sl in enumerate(slots):
+        marks[i][0].record()
+        for l in range(L):
+            tq.tq_append_kv(lay, True, kn[i, l], kp[l], N, sl, Pi, cd, td, S=S, positions=kpos[i], rope_base=base,
+                            d_status=status)
+            tq.tq_append_kv(lay, False, vn[i, l], vp[l], N, sl, Pi, cd, td, d_status=status)
+            if l == 0:
+                marks[i][1].record()
+            tq.tq_decode_attention(lay, Q[l], kp[l], vp[l], HKV, sl + 1, Pi, Pi, S, cd, cd, out[l], ws,
+                                   q_positions=qpos[i], rope_base=base, ctx_stride=N, d_status=status)
+        marks[i][2].record()
+    torch.cuda.synchronize()
+    launches = tq.tq_kernel_launches() - n0
+    barrier(world)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    per_token = max_over_ranks(world, statistics.mean(m[0].elapsed_time(m[2]) for m in marks))
+    append_l0 = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    return {"us_per_generated_token": 1e3 * per_token, "tokens_per_s": world * B / (per_token * 1e-3),
+            "layers": L, "steps": T, "append_us_layer0": 1e3 * append_l0, "gpu_launches": launches,
+            "note": (f"per step and layer: tq_append_kv of {streams} keys (RoPE) and {streams} values at slot "
+                     f"N-{T}+i, then tq_decode_attention over slot+1 tokens (ctx_stride {N}); "
+                     f"tokens_per_s counts the batch's {B} sequences")}
 
 
 def run_e2e_c3(args, tq, lay, K, V, Q, kp, vp, out, ws, Pi, S, cd, td, status, shape, world):
@@ -1053,6 +1136,16 @@ def run_c5(args, world, rank, tq):
     torch.backends.cuda.matmul.allow_tf32 = prev
     got = top_i.cpu().numpy()
     recall = float(np.mean([len(set(a.tolist()) & set(b.tolist())) for a, b in zip(got, exact)]) / k)
+    # The pages' measure, recall 1@k: how often the true best inner product
+    # is among the first k estimated results (one untimed call with k = 32).
+    k32 = 32
+    ti32 = torch.empty((nq, k32), dtype=torch.int64, device=dev)
+    ts32 = torch.empty((nq, k32), dtype=torch.float32, device=dev)
+    ws32 = torch.empty(tq.tq_search_workspace_bytes(lay, nq, n_db, k32) + 256, dtype=torch.uint8, device=dev)
+    tq.tq_search_topk(lay, Qd, planes, n_db, Pi, S, cd, k32, ti32, ts32, ws32)
+    g32 = ti32.cpu().numpy()
+    assert np.array_equal(g32[:, :k], got), "top-10 is the head of top-32"
+    one_at = {str(kk): float(np.mean([exact[r, 0] in g32[r, :kk] for r in range(nq)])) for kk in (1, 2, 4, 8, 16, 32)}
     # Work per estimated score at head_dim d, in FP32 lane ops: d adds of the
     # per-coordinate code table, d/4 adds of the sign-nibble table, 2 for the
     # norm-weighted combination.
@@ -1065,6 +1158,7 @@ def run_c5(args, world, rank, tq):
                        "l2": "L2 flushed (384 MiB write) before every timed call; only the calls are timed"},
                       T.clk, T.launches)
     res["recall_at_10"] = recall
+    res["recall_1_at_k"] = one_at
     res["recall_reference"] = "exact fp32 inner-product top-10 of all 10,000 queries (torch matmul, TF32 off)"
     res["index_build"] = {"quantize_us": 1e3 * build_ms, "vectors_per_s": n_db / (build_ms * 1e-3),
                           "roofline": hbm_roofline("tq_quantize_kv(d=200 fp32 keys): quantize_kernel<200>",

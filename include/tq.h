@@ -158,7 +158,7 @@ tq_status tq_make_codebook(int32_t d, int32_t bits, int32_t mode,
  *  centroids, boundaries   device float, 2^bits and 2^bits-1 entries
  *  out             planes to write, n_vectors rows each (pointers device)
  *  d_status        device int32 (nullable), see TQ_DEV_*
- * Supported d: 64, 128, 200 (and other multiples of 8 up to 256).
+ * Supported d: 64, 128, 200 (others: TQ_ERR_UNSUPPORTED).
  * ---------------------------------------------------------------------- */
 tq_status tq_quantize_kv(const tq_layout* layout, int32_t is_key,
                          const void* x, tq_dtype x_dtype, int64_t n_vectors, int64_t row_stride,
@@ -168,6 +168,35 @@ tq_status tq_quantize_kv(const tq_layout* layout, int32_t is_key,
                          const float* centroids, const float* boundaries,
                          const tq_planes* out,
                          int32_t* d_status, void* stream);
+
+/* ------------------------------------------------------------------------
+ * tq_append_kv — quantise one new vector per stream into its cache slot
+ * (one launch; device).
+ *
+ * 7minutos.es "KV cache ... TurboQuant" Etapa 1: a token's indices are
+ * computed once, when it enters the cache, and stay there until it is
+ * evicted; gist.science TurboESM section 2A: RoPE at the token's position
+ * before the rotation. The arithmetic is that of tq_quantize_kv with one
+ * shared Pi; only the destination differs: row s of x (stream s = b * hkv +
+ * kv) is written to cache row s * ctx_stride + slot, the layout that
+ * tq_decode_attention reads with the same ctx_stride.
+ *
+ *  x            device, n_streams rows of d elements (TQ_F32 or TQ_BF16),
+ *               row s at x + s*row_stride elements
+ *  positions    device int32 [n_streams] RoPE positions, or NULL (no RoPE)
+ *  Pi, S        device float d x d (S: keys only)
+ *  cache        planes of n_streams * ctx_stride rows (device pointers)
+ *  slot         0 <= slot < ctx_stride; rows at other slots are not touched
+ * Errors: TQ_ERR_INVALID_ARG (NULL pointers, slot out of range, strides),
+ * TQ_ERR_UNSUPPORTED (d not 64, 128 or 200), TQ_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+tq_status tq_append_kv(const tq_layout* layout, int32_t is_key,
+                       const void* x, tq_dtype x_dtype, int64_t n_streams, int64_t row_stride,
+                       const int32_t* positions, float rope_base,
+                       const float* Pi, const float* S,
+                       const float* centroids, const float* boundaries,
+                       const tq_planes* cache, int64_t ctx_stride, int64_t slot,
+                       int32_t* d_status, void* stream);
 
 /* ------------------------------------------------------------------------
  * tq_decode_attention — attention of queries over a packed K/V cache.

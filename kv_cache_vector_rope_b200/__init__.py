@@ -58,6 +58,8 @@ _SIGNATURES = {
     "tq_decode_attention": (ctypes.c_int, [ctypes.POINTER(Layout), _P, ctypes.c_int, _I32, _I32, _I32, _I32, _I64,
                                            _I64, _P, _F32, ctypes.POINTER(_Planes), ctypes.POINTER(_Planes),
                                            _P, _P, _I64, _P, _P, _P, _F32, _P, ctypes.c_int, _P, _P, _SZ, _P, _P]),
+    "tq_append_kv": (ctypes.c_int, [ctypes.POINTER(Layout), _I32, _P, ctypes.c_int, _I64, _I64, _P, _F32, _P, _P, _P, _P,
+                                    ctypes.POINTER(_Planes), _I64, _I64, _P, _P]),
     "tq_decode_workspace_bytes": (_SZ, [ctypes.POINTER(Layout), _I32, _I32, _I32, _I32, _I64]),
     "tq_decode_attention_noalloc": (ctypes.c_int, [ctypes.POINTER(Layout), _P, ctypes.c_int, _I32, _I32, _I32, _I32,
                                                    _I64, _I64, _P, _F32, ctypes.POINTER(_Planes),
@@ -204,6 +206,19 @@ def tq_quantize_kv(lay: Layout, is_key: bool, x: torch.Tensor, out: Planes, Pi: 
                                x.stride(0), _ptr(positions), float(rope_base), _dev(Pi, "Pi"), vectors_per_pi,
                                pi_stride, _ptr(S), _dev(centroids, "centroids"), _dev(boundaries, "boundaries"),
                                ctypes.byref(out.c()), _ptr(d_status), _stream(stream)))
+
+
+def tq_append_kv(lay: Layout, is_key: bool, x: torch.Tensor, cache: Planes, ctx_stride: int, slot: int,
+                 Pi: torch.Tensor, centroids: torch.Tensor, boundaries: torch.Tensor, S: torch.Tensor | None = None,
+                 positions: torch.Tensor | None = None, rope_base: float = 0.0, d_status: torch.Tensor | None = None,
+                 stream=None) -> None:
+    """Quantises row s of x ([n_streams, d]) into cache row s * ctx_stride + slot."""
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be [n_streams, d] with unit stride along d")
+    _check(_lib.tq_append_kv(ctypes.byref(lay), int(is_key), _dev(x, "x"), _dtype_code(x), x.shape[0], x.stride(0),
+                             _ptr(positions), float(rope_base), _dev(Pi, "Pi"), _ptr(S), _dev(centroids, "centroids"),
+                             _dev(boundaries, "boundaries"), ctypes.byref(cache.c()), ctx_stride, slot,
+                             _ptr(d_status), _stream(stream)))
 
 
 def tq_decode_workspace_bytes(lay: Layout, batch: int, hq: int, hkv: int, nq: int, n_ctx: int) -> int:

@@ -408,8 +408,9 @@ extern "C" tq_status tq_quantize_kv(const tq_layout* layout, int32_t is_key, con
               out->idx, is_key ? out->sign : nullptr, out->norm, is_key ? out->rnorm : nullptr, d_status};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool rope = positions != nullptr && rope_base > 0.f;
-  if (!getenv_force_cuda_core() && tc_quantize_supported(d, x_dtype, rope, pi_stride, x, row_stride))
-    return tc_quantize(d, is_key != 0, bits, x, n_vectors, row_stride, Pi, S, centroids, boundaries, out, d_status, s);
+  if (!getenv_force_cuda_core() && tc_quantize_supported(d, x_dtype, rope, vectors_per_pi, pi_stride, x, row_stride))
+    return tc_quantize(d, is_key != 0, bits, x, n_vectors, row_stride, Pi, vectors_per_pi, pi_stride, S, centroids,
+                       boundaries, out, d_status, s);
   cudaError_t e;
   switch (d) {
     case 64: e = launch<64>(a, s); break;
@@ -420,3 +421,4 @@ extern "C" tq_status tq_quantize_kv(const tq_layout* layout, int32_t is_key, con
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_quantize_kv launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }
+

@@ -72,7 +72,7 @@ constexpr int pow2_at_least(int x) {
   return p;
 }
 
-template <int D, bool KEY>
+template <int D, bool KEY, bool PH = false>
 struct Cfg {
   static constexpr int kM = 128;
   static constexpr int kKSteps = D / 16;
@@ -86,12 +86,16 @@ struct Cfg {
   static constexpr int kTmemCols = pow2_at_least(2 * kSlotCols);
   static constexpr int kChunks = D / 32;             // 32-column chunks
   // Shared memory plan (offsets from a 1024-aligned base).
+  // Pi splits: one slot, or two (per-head mode: the next head's Pi is
+  // written into the other slot while the current one is in use).
+  static constexpr int kPiSlot = 3 * kMatBytes;
   static constexpr int kOffPi = 0;
-  static constexpr int kOffS = kOffPi + 3 * kMatBytes;
+  static constexpr int kOffS = kOffPi + (PH ? 2 : 1) * kPiSlot;
   static constexpr int kOffX = kOffS + kSSplits * kMatBytes;
   static constexpr int kOffBar = kOffX + kStages * kTileBytes;
-  // full[st], empty[st], yfull[2], rfull[2], pfull[2], accfree[2], drain
-  static constexpr int kNumBars = 2 * kStages + 8 + 1;
+  // full[st], empty[st], yfull[2], rfull[2], pfull[2], accfree[2], drain,
+  // pi_full[2], pi_free[2]
+  static constexpr int kNumBars = 2 * kStages + 8 + 1 + 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   // misc: tmem base (4) + abort (4) + r-scale exponent shift (4) + symmetric-table flag (4) + cent[16] + bnd[16]
   static constexpr int kOffCent = kOffMisc + 16;
@@ -113,6 +117,8 @@ struct TcArgs {
   float* rnorm;
   int32_t* d_status;
   uint64_t wait_ns;     // pipeline wait limit (drains keep 2 s)
+  int64_t vpp;          // vectors per rotation (per-head mode)
+  int64_t pi_stride;    // floats between rotations; 0: one shared Pi
 };
 
 // Splits v into bf16 terms hi + mid + lo that add up to v to ~2^-25.
@@ -180,9 +186,29 @@ __device__ __forceinline__ int code_symmetric3(float y, const float (&th)[NB], f
   return (y > 0.f ? 4 : 3) ^ m;
 }
 
-template <int D, bool KEY, int BITS>
+// bf16 splits hi + mid + lo of Pi into one slot (three K-major, 128B-swizzled
+// matrices), elements first, first + step, ...
+template <int D>
+__device__ __forceinline__ void stage_pi3(unsigned char* slot, const float* __restrict__ Pi, int first, int step) {
+  constexpr int kMat = D * D * 2;
+#pragma unroll 4
+  for (int e = first; e < D * D; e += step) {
+    const uint32_t off = sw128_offset(e / D, e % D, D);
+    __nv_bfloat16 h, m, l;
+    split3(__ldg(Pi + e), h, m, l);
+    *reinterpret_cast<__nv_bfloat16*>(slot + off) = h;
+    *reinterpret_cast<__nv_bfloat16*>(slot + kMat + off) = m;
+    *reinterpret_cast<__nv_bfloat16*>(slot + 2 * kMat + off) = l;
+  }
+}
+
+// PH (per-head mode, d = 64): vector v uses Pi + (v / vpp) pi_stride, with vpp
+// a multiple of the 128-vector tile. Each CTA then takes a contiguous range of
+// tiles, and the producer warp writes each new head's Pi splits into the slot
+// the head before last used (pi_free), announcing them with pi_full.
+template <int D, bool KEY, int BITS, bool PH>
 __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcArgs a) {
-  using C = Cfg<D, KEY>;
+  using C = Cfg<D, KEY, PH>;
   constexpr int kNb = (1 << BITS) - 1;
   constexpr int kRowBytes = D * BITS / 8;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -198,6 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
   uint64_t* pfull = rfull + 2;                        // [2]
   uint64_t* accfree = pfull + 2;                      // [2]
   uint64_t* drain = accfree + 2;                      // [1] final MMA drain
+  uint64_t* pi_full = drain + 1;                      // [2] per-head mode: Pi slot written
+  uint64_t* pi_free = pi_full + 2;                    // [2] per-head mode: MMAs done with the slot
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
   volatile int* abort_s = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
   int* rshift_s = reinterpret_cast<int*>(sm + C::kOffMisc + 8);
@@ -207,7 +235,14 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_tiles = (a.n + C::kM - 1) / C::kM;
-  const int my_tiles = (n_tiles > blockIdx.x) ? static_cast<int>((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+  // Tiles of this CTA: every gridDim.x-th (shared Pi), or a contiguous range
+  // (per-head mode: few head changes per CTA).
+  const int64_t ph_lo = n_tiles * blockIdx.x / gridDim.x, ph_hi = n_tiles * (blockIdx.x + 1) / gridDim.x;
+  const int my_tiles = PH ? static_cast<int>(ph_hi - ph_lo)
+                          : (n_tiles > blockIdx.x) ? static_cast<int>((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x)
+                                                   : 0;
+  auto tile_of = [&](int it) -> int64_t { return PH ? ph_lo + it : blockIdx.x + int64_t(it) * gridDim.x; };
+  auto head_of = [&](int64_t t) -> int64_t { return PH ? t * C::kM / a.vpp : 0; };
 
   // ---------------------------------------------------------------- prologue
   if (tid == 0) {
@@ -222,6 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       mbar_init(&accfree[b], 4);
     }
     mbar_init(drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pi_full[b], 1);
+      mbar_init(&pi_free[b], 1);
+    }
     *abort_s = 0;
     // r 2^k must stay below 2^14 for fp16: |r| <= (1 + max|c|) ||y||.
     float lim = 1.f;
@@ -244,15 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     tmem_alloc(tmem_base_s, C::kTmemCols);
     tmem_relinquish();
   }
-  // bf16 splits of Pi (3) and fp16 splits of S (2), K-major, 128B-swizzled.
+  // bf16 splits of Pi (3) and fp16 splits of S (2), K-major, 128B-swizzled
+  // (per-head mode: the producer stages each head's Pi).
+  if (!PH) stage_pi3<D>(pi_s, a.Pi, tid, kThreads);
   for (int e = tid; e < D * D; e += kThreads) {
     const int i = e / D, j = e % D;
     const uint32_t off = sw128_offset(i, j, D);
-    __nv_bfloat16 h, m, l;
-    split3(__ldg(a.Pi + e), h, m, l);
-    *reinterpret_cast<__nv_bfloat16*>(pi_s + off) = h;
-    *reinterpret_cast<__nv_bfloat16*>(pi_s + C::kMatBytes + off) = m;
-    *reinterpret_cast<__nv_bfloat16*>(pi_s + 2 * C::kMatBytes + off) = l;
     if (KEY) {
       const float sv = __ldg(a.S + e);
       const __half sh = __float2half_rn(sv);
@@ -278,22 +314,53 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      int armed[C::kStages];
-      for (int s = 0; s < C::kStages; ++s) armed[s] = 0;
-      for (int it = 0; it < my_tiles; ++it) {
-        const int64_t t = blockIdx.x + int64_t(it) * gridDim.x;
+    // The whole warp runs the loop (it stages the per-head Pi splits); lane 0
+    // issues the tile loads.
+    int armed[C::kStages];
+    for (int s = 0; s < C::kStages; ++s) armed[s] = 0;
+    int64_t cur_head = -1;
+    int nh = 0;                                   // heads staged so far
+    for (int it = 0; it < my_tiles; ++it) {
+      const int64_t t = tile_of(it);
+      if (PH) {
+        const int64_t h = head_of(t);
+        if (h != cur_head) {
+          const int slot = nh & 1;
+          bool ok = *abort_s == 0;
+          if (ok && nh >= 2) ok = mbar_wait(&pi_free[slot], ((nh - 2) >> 1) & 1, a.wait_ns);
+          if (!__all_sync(0xffffffffu, ok)) {
+            if (lane == 0 && !*abort_s) fail();
+            break;
+          }
+          stage_pi3<D>(pi_s + slot * C::kPiSlot, a.Pi + h * a.pi_stride, lane, 32);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pi_full[slot]);
+          cur_head = h;
+          ++nh;
+        }
+      }
+      int go = 1;
+      if (lane == 0) {
         const int st = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
-        if (*abort_s) break;
-        if (!mbar_wait(&empty[st], ph ^ 1, a.wait_ns)) { fail(); break; }
-        mbar_expect_tx(&full[st], C::kTileBytes);
-        unsigned char* dst = x_s + st * C::kTileBytes;
+        if (*abort_s) {
+          go = 0;
+        } else if (!mbar_wait(&empty[st], ph ^ 1, a.wait_ns)) {
+          fail();
+          go = 0;
+        } else {
+          mbar_expect_tx(&full[st], C::kTileBytes);
+          unsigned char* dst = x_s + st * C::kTileBytes;
 #pragma unroll
-        for (int k = 0; k < D / 64; ++k) tma_load_2d(dst + k * C::kM * 128, &tmap, &full[st], k * 64, int(t * C::kM));
-        armed[st] = it + 1;
+          for (int k = 0; k < D / 64; ++k) tma_load_2d(dst + k * C::kM * 128, &tmap, &full[st], k * 64, int(t * C::kM));
+          armed[st] = it + 1;
+        }
       }
-      // Never leave a copy in flight: wait for the last load of every stage.
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+    }
+    // Never leave a copy in flight: wait for the last load of every stage.
+    if (lane == 0) {
       for (int s = 0; s < C::kStages; ++s) {
         if (armed[s]) mbar_wait(&full[s], ((armed[s] - 1) / C::kStages) & 1);
       }
@@ -305,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
       constexpr uint32_t kIdescP = (1u << 4) | (static_cast<uint32_t>(D >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
       const uint64_t pi_desc0 = desc_k_sw128(smem_u32(pi_s)), s_desc0 = desc_k_sw128(smem_u32(s_s)),
                      x_desc0 = desc_k_sw128(smem_u32(x_s));
-      auto issue_y = [&](int it) {
+      auto issue_y = [&](int it, int pslot) {
         const int st = it % C::kStages;
         const int b = it & 1;
         const uint32_t d_tmem = tmem + b * C::kSlotCols;
@@ -319,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           for (int k = 0; k < C::kKSteps; ++k) {
             constexpr int kAtomA = 128 * 128, kAtomB = D * 128;
             const uint64_t ad = xa + static_cast<uint64_t>(((k >> 2) * kAtomA + (k & 3) * 32) >> 4);
-            const uint64_t bd = pi_desc0 + static_cast<uint64_t>((sp * C::kMatBytes + (k >> 2) * kAtomB + (k & 3) * 32) >> 4);
+            const uint64_t bd = pi_desc0 + static_cast<uint64_t>(
+                                               (pslot * C::kPiSlot + sp * C::kMatBytes + (k >> 2) * kAtomB + (k & 3) * 32) >> 4);
             umma_ss(d_tmem, ad, bd, kIdescY, (q | k) != 0);
           }
         }
@@ -344,6 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
         umma_commit(&pfull[b]);
       };
       int ny = 0, np = 0;
+      int64_t icur = -1;                         // per-head mode: head of the last issued tile
+      int inh = 0;                               // heads issued so far
       uint64_t last = globaltimer_ns();
       while (KEY ? (np < my_tiles) : (ny < my_tiles)) {
         if (*abort_s) break;
@@ -352,9 +422,19 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
           const int st = ny % C::kStages;
           const uint32_t ph = (ny / C::kStages) & 1;
           const uint32_t bph = (ny >> 1) & 1;
-          if (mbar_try_wait(&full[st], ph) && mbar_try_wait(&accfree[ny & 1], bph ^ 1)) {
+          const int64_t h = head_of(tile_of(ny));
+          const int nh_t = (PH && h != icur) ? inh + 1 : inh;   // heads including this tile's
+          const int pslot = PH ? (nh_t - 1) & 1 : 0;
+          const bool pi_ok = !PH || h == icur || mbar_try_wait(&pi_full[pslot], ((nh_t - 1) >> 1) & 1);
+          if (pi_ok && mbar_try_wait(&full[st], ph) && mbar_try_wait(&accfree[ny & 1], bph ^ 1)) {
             tc_fence_after();
-            issue_y(ny);
+            issue_y(ny, pslot);
+            if (PH) {
+              icur = h;
+              inh = nh_t;
+              // The head's last tile: its Pi slot is free once these MMAs complete.
+              if (ny + 1 == my_tiles || head_of(tile_of(ny + 1)) != h) umma_commit(&pi_free[pslot]);
+            }
             ++ny;
             progress = true;
           }
@@ -386,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
     const bool sym = *sym_s != 0;
     float th[kNb];
     for (int it = wg; it < my_tiles; it += 2) {
-      const int64_t t = blockIdx.x + int64_t(it) * gridDim.x;
+      const int64_t t = tile_of(it);
       const uint32_t ph = (it >> 1) & 1;
       const int64_t v = t * C::kM + row;
       const bool valid = v < a.n;
@@ -722,7 +802,9 @@ __device__ __forceinline__ void fix_batch(const TcArgs& a, const int64_t (&rows)
   __syncwarp();                                          // scratch reused by the next batch
 }
 
-template <int D, bool KEY, int BITS>
+// Per-head mode: a window never crosses a head, and Pi^T is staged again
+// when a window with flagged rows belongs to another head than the last.
+template <int D, bool KEY, int BITS, bool PH>
 __global__ void __launch_bounds__(kFixThreads, 1) quantize_fixup(TcArgs a) {
   using F = FixCfg<D, KEY>;
   extern __shared__ __align__(16) unsigned char fix_smem[];
@@ -742,8 +824,14 @@ __global__ void __launch_bounds__(kFixThreads, 1) quantize_fixup(TcArgs a) {
   const int64_t r0 = int64_t(blockIdx.x) * per;
   const int64_t r1 = r0 + per < a.n ? r0 + per : a.n;
   bool staged = false;
-  for (int64_t w0 = r0; w0 < r1; w0 += kFixList) {
-    const int64_t w1 = w0 + kFixList < r1 ? w0 + kFixList : r1;
+  int64_t staged_head = -1;
+  int64_t w1 = r0;
+  for (int64_t w0 = r0; w0 < r1; w0 = w1) {
+    w1 = w0 + kFixList < r1 ? w0 + kFixList : r1;
+    if (PH) {
+      const int64_t hb = (w0 / a.vpp + 1) * a.vpp;          // next head boundary
+      if (hb < w1) w1 = hb;
+    }
     if (threadIdx.x == 0) {
       cnt = 0;
       taken = 0;
@@ -766,11 +854,13 @@ __global__ void __launch_bounds__(kFixThreads, 1) quantize_fixup(TcArgs a) {
     __syncthreads();
     const int total = cnt;
     if (total == 0) continue;
-    if (!staged) {
-      stage_transposed<D>(PiT, a.Pi);
-      if (KEY) stage_transposed<D>(ST, a.S);
+    const int64_t head = PH ? w0 / a.vpp : 0;
+    if (!staged || head != staged_head) {
+      stage_transposed<D>(PiT, a.Pi + head * a.pi_stride);
+      if (KEY && !staged) stage_transposed<D>(ST, a.S);
       __syncthreads();
       staged = true;
+      staged_head = head;
     }
     for (;;) {
       int e = 0;
@@ -805,55 +895,59 @@ EncodeFn encode_fn() {
   return fn;
 }
 
-template <int D, bool KEY, int BITS>
+template <int D, bool KEY, int BITS, bool PH>
 cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& map, cudaStream_t st) {
-  using C = Cfg<D, KEY>;
+  using C = Cfg<D, KEY, PH>;
   static_assert(C::kSmemBytes <= 232448, "shared memory plan exceeds 227 KB");
-  cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<D, KEY, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(quantize_tc_kernel<D, KEY, BITS, PH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = (a.n + 127) / 128;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  quantize_tc_kernel<D, KEY, BITS><<<grid, kThreads, C::kSmemBytes, st>>>(map, a);
+  quantize_tc_kernel<D, KEY, BITS, PH><<<grid, kThreads, C::kSmemBytes, st>>>(map, a);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   constexpr size_t fix_smem = FixCfg<D, KEY>::kBytes;
   static_assert(FixCfg<D, KEY>::kBytes <= 232448, "fixup shared memory plan exceeds 227 KB");
-  e = cudaFuncSetAttribute(quantize_fixup<D, KEY, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(quantize_fixup<D, KEY, BITS, PH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(fix_smem));
   if (e != cudaSuccess) return e;
   const int64_t fix_ctas = (a.n + kFixList - 1) / kFixList;
-  quantize_fixup<D, KEY, BITS><<<static_cast<int>(fix_ctas < sms ? (fix_ctas < 1 ? 1 : fix_ctas) : sms), kFixThreads,
-                                 fix_smem, st>>>(a);
+  quantize_fixup<D, KEY, BITS, PH><<<static_cast<int>(fix_ctas < sms ? (fix_ctas < 1 ? 1 : fix_ctas) : sms),
+                                     kFixThreads, fix_smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }
 
-template <int D, bool KEY>
+template <int D, bool KEY, bool PH = false>
 cudaError_t launch_bits(int bits, const TcArgs& a, const CUtensorMap& map, cudaStream_t st) {
   switch (bits) {
-    case 2: return launch_tc<D, KEY, 2>(a, map, st);
-    case 3: return launch_tc<D, KEY, 3>(a, map, st);
-    default: return launch_tc<D, KEY, 4>(a, map, st);
+    case 2: return launch_tc<D, KEY, 2, PH>(a, map, st);
+    case 3: return launch_tc<D, KEY, 3, PH>(a, map, st);
+    default: return launch_tc<D, KEY, 4, PH>(a, map, st);
   }
 }
 
 }  // namespace
 
-bool tc_quantize_supported(int d, int x_dtype, bool rope, int64_t pi_stride, const void* x, int64_t row_stride) {
+bool tc_quantize_supported(int d, int x_dtype, bool rope, int64_t vectors_per_pi, int64_t pi_stride, const void* x,
+                           int64_t row_stride) {
   if (!(d == 64 || d == 128)) return false;
-  if (x_dtype != TQ_BF16 || rope || pi_stride != 0) return false;
+  if (x_dtype != TQ_BF16 || rope) return false;
+  // Per-head rotations: d = 64 (two Pi slots fit beside the pipeline), and no
+  // 128-vector tile may straddle two heads.
+  if (pi_stride != 0 && !(d == 64 && vectors_per_pi > 0 && vectors_per_pi % 128 == 0)) return false;
   if (!aligned(x, 16) || (row_stride * 2) % 16 != 0) return false;
   return encode_fn() != nullptr;
 }
 
 tq_status tc_quantize(int d, bool is_key, int bits, const void* x, int64_t n, int64_t row_stride, const float* Pi,
-                      const float* S, const float* cent, const float* bnd, const tq_planes* out, int32_t* d_status,
-                      cudaStream_t st) {
+                      int64_t vectors_per_pi, int64_t pi_stride, const float* S, const float* cent, const float* bnd,
+                      const tq_planes* out, int32_t* d_status, cudaStream_t st) {
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride) * 2};
@@ -864,10 +958,13 @@ tq_status tc_quantize(int d, bool is_key, int bits, const void* x, int64_t n, in
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   TcArgs a{static_cast<const __nv_bfloat16*>(x), n, row_stride, Pi, S, cent, bnd, out->idx,
-           is_key ? out->sign : nullptr, out->norm, is_key ? out->rnorm : nullptr, d_status, pipeline_wait_ns()};
+           is_key ? out->sign : nullptr, out->norm, is_key ? out->rnorm : nullptr, d_status, pipeline_wait_ns(),
+           pi_stride != 0 ? vectors_per_pi : 1, pi_stride};
   cudaError_t e;
   if (d == 128)
     e = is_key ? launch_bits<128, true>(bits, a, map, st) : launch_bits<128, false>(bits, a, map, st);
+  else if (pi_stride != 0)
+    e = is_key ? launch_bits<64, true, true>(bits, a, map, st) : launch_bits<64, false, true>(bits, a, map, st);
   else
     e = is_key ? launch_bits<64, true>(bits, a, map, st) : launch_bits<64, false>(bits, a, map, st);
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tensor-core quantize launch: %s", cudaGetErrorString(e));

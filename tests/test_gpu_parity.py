@@ -427,3 +427,30 @@ def test_output_fences_intact_after_quantize_decode_dequantize():
     bufs += [ob, wb, sb, db]
     assert all(_fences_intact(b) for b in bufs)
     assert torch.isfinite(out).all() and torch.isfinite(deq).all()
+
+
+# ---------------------------------------------------------------------------
+# Per-head rotations (one Pi per `vpp` consecutive vectors): the tensor-core
+# quantiser takes them at d = 64 when vpp is a multiple of its 128-vector
+# tile (many heads per CTA, so the two Pi slots are reused), the CUDA-core
+# kernel otherwise (vpp = 100). Ragged last head in every case.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("vpp,heads", [(128, 600), (384, 100), (100, 50)])
+def test_per_head_rotation_quantize(bits, vpp, heads):
+    d = 64
+    n = heads * vpp - 37
+    rg = np.random.default_rng(1000 * bits + vpp)
+    X = rg.standard_normal((n, d))
+    X[:, rg.choice(d, 4, replace=False)] *= 8.0
+    X[7] = 0.0
+    Xb = synth.to_bf16(X.astype(np.float32))
+    X64 = Xb.float().numpy().astype(np.float64)
+    Pis = np.stack([synth.random_rotation(d, 50 + h) for h in range(heads)])
+    S = synth.gaussian_projection(d, 4)
+    group = np.arange(n) // vpp
+    for is_key in (True, False):
+        planes = quantize_gpu(Xb.cuda(), d, bits, is_key, Pis.reshape(heads * d, d), S if is_key else None,
+                              vpp=vpp, pi_stride=d * d)
+        ref = quantize_ref(X64, d, bits, is_key, Pis, S if is_key else None, pi_group=group)
+        P.compare_quantized(P.host_planes(planes), ref, d, bits, is_key)

@@ -128,6 +128,27 @@ def test_quantize_host_validation():
     assert _raw_quantize(lay, is_key=1, planes=tq._Planes(0x6000, 0, 0x8000, 0x9000)) == tq.TQ_ERR_INVALID_ARG
 
 
+def _raw_append(lay, is_key=1, x=0x1000, n=4, row_stride=128, Pi=0x2000, S=0x3000, ctx_stride=100, slot=7,
+                planes=None):
+    planes = planes or tq._Planes(0x6000, 0x7000, 0x8000, 0x9000)
+    return tq._lib.tq_append_kv(ctypes.byref(lay), is_key, x, 0, n, row_stride, None, 0.0, Pi, S, 0x4000, 0x5000,
+                                ctypes.byref(planes), ctx_stride, slot, None, None)
+
+
+def test_append_host_validation():
+    lay = tq.layout(128, 3, 3)
+    assert _raw_append(lay, n=0) == tq.TQ_OK             # nothing to do, nothing launched
+    assert _raw_append(lay, n=-1) == tq.TQ_ERR_INVALID_ARG
+    assert _raw_append(lay, slot=100) == tq.TQ_ERR_INVALID_ARG      # slot must be < ctx_stride
+    assert "slot" in tq.tq_last_error_string()
+    assert _raw_append(lay, slot=-1) == tq.TQ_ERR_INVALID_ARG
+    assert _raw_append(lay, ctx_stride=0, slot=0) == tq.TQ_ERR_INVALID_ARG
+    assert _raw_append(lay, S=0) == tq.TQ_ERR_INVALID_ARG
+    assert _raw_append(lay, row_stride=100) == tq.TQ_ERR_INVALID_ARG
+    assert _raw_append(lay, Pi=0x2004) == tq.TQ_ERR_INVALID_ARG
+    assert _raw_append(tq.layout(96, 3, 3), row_stride=96) == tq.TQ_ERR_UNSUPPORTED
+
+
 def _raw_decode(lay, hq=32, hkv=8, nq=1, n_ctx=1024, ctx_stride=0, ws=0x10000, ws_bytes=1 << 30, kp=None):
     kp = kp or tq._Planes(0x1000, 0x2000, 0x3000, 0x4000)
     vp = tq._Planes(0x5000, 0, 0x6000, 0)
