@@ -635,12 +635,107 @@ def esm_setup(tq, seed, dev):
     uv = np.concatenate([tq.tq_rotate_normalize(cV[l, h], PiV[l * H + h]).ravel() for l in range(L) for h in range(H)])
     ck, tk, _ = tq.tq_make_codebook(d, 3, 1, uk)
     cv, tv, _ = tq.tq_make_codebook(d, 3, 1, uv)
-    return data, PiK, PiV, (ck, tk), (cv, tv)
+    return data, PiK, PiV, (ck, tk), (cv, tv), (uk, uv)
+
+
+def variants_c2(tq, data, PiK_h, PiV_h, books, samples, dev, layer=7):
+    """Layout and correction variants on one layer of the ESM-shaped cache (untimed, evaluation only).
+
+    Reconstructions (library kernels) against the bf16 inputs, scores q.k/sqrt(d) and softmax outputs of all
+    1024 queries per head against fp32 attention on the inputs (torch, as the measuring stick):
+      qjl        3-bit codes + QJL signs of S r + ||r|| (the configs' keys; tq_dequantize)
+      sign_mean  3-bit codes + signs of r itself + ||x||, corrected by e_bar (TurboESM; S = I)
+      plain      3-bit codes + ||x|| (the configs' values)
+      b-1+1      TurboQuant's budget at b = 3: 2-bit codes + QJL (keys)
+      shared     one table fitted on K and V samples pooled, instead of one each (dual)"""
+    (ck, tk), (cv, tv) = books
+    uk, uv = samples
+    L, H, N, d = data.K.shape
+    rows = slice(layer * H * N, (layer + 1) * H * N)
+    n = H * N
+    K = data.K.reshape(-1, d)[rows].to(dev)
+    V = data.V.reshape(-1, d)[rows].to(dev)
+    Q = data.Q[layer].to(dev).float()                                   # [H, N, d]
+    PiK = torch.as_tensor(PiK_h[layer * H:(layer + 1) * H], device=dev).reshape(H * d, d).contiguous()
+    PiV = torch.as_tensor(PiV_h[layer * H:(layer + 1) * H], device=dev).reshape(H * d, d).contiguous()
+    S = torch.as_tensor(data.S, device=dev)
+    eye = torch.eye(d, device=dev)
+    lay3 = tq.layout(d, 3, 3)
+    cs, ts, _ = tq.tq_make_codebook(d, 3, 1, np.concatenate([uk, uv]))
+    ck2, tk2, _ = tq.tq_make_codebook(d, 2, 1, uk)
+    e_k = tq.tq_residual_mean(uk, ck, tk, 3)
+    e_v = tq.tq_residual_mean(uv, cv, tv, 3)
+    T = lambda a: torch.as_tensor(np.ascontiguousarray(a), device=dev, dtype=torch.float32)
+
+    def quant(x, Pi, c, t, bits, Sm):
+        lay = tq.layout(d, bits, bits)
+        p = tq.alloc_planes(n, d, bits, Sm is not None, dev)
+        tq.tq_quantize_kv(lay, Sm is not None, x, p, Pi, T(c), T(t), S=Sm, vectors_per_pi=N, pi_stride=d * d)
+        return lay, p
+
+    def deq(lay, p, Pi, c, mode, e=0.0):
+        o = torch.empty((n, d), device=dev)
+        if mode == "qjl":
+            tq.tq_dequantize(lay, True, p, n, Pi, T(c), o, S=S, vectors_per_pi=N, pi_stride=d * d)
+        elif mode == "sign_mean":
+            tq.tq_dequantize_sign_mean(lay, True, p, n, Pi, T(c), e, o, vectors_per_pi=N, pi_stride=d * d)
+        else:
+            tq.tq_dequantize(lay, False, p, n, Pi, T(c), o, vectors_per_pi=N, pi_stride=d * d)
+        return o
+
+    lk, pk = quant(K, PiK, ck, tk, 3, S)
+    lki, pki = quant(K, PiK, ck, tk, 3, eye)
+    lvi, pvi = quant(V, PiV, cv, tv, 3, eye)
+    lk2, pk2 = quant(K, PiK, ck2, tk2, 2, S)
+    lks, pks = quant(K, PiK, cs, ts, 3, None)
+    lvs, pvs = quant(V, PiV, cs, ts, 3, None)
+    rec = {
+        "K": {"plain": deq(lk, pk, PiK, ck, "plain"), "qjl": deq(lk, pk, PiK, ck, "qjl"),
+              "sign_mean": deq(lki, pki, PiK, ck, "sign_mean", e_k), "b-1+1": deq(lk2, pk2, PiK, ck2, "qjl"),
+              "plain_shared": deq(lks, pks, PiK, cs, "plain")},
+        "V": {"plain": deq(lvi, pvi, PiV, cv, "plain"), "sign_mean": deq(lvi, pvi, PiV, cv, "sign_mean", e_v),
+              "plain_shared": deq(lvs, pvs, PiV, cs, "plain")},
+    }
+    torch.cuda.synchronize()
+    Kf, Vf = K.float(), V.float()
+
+    def snr(x, y):
+        return float(10 * torch.log10((x * x).sum() / ((x - y) ** 2).sum()))
+
+    out = {"e_bar": {"K": e_k, "V": e_v}, "snr_db": {t_: {m: snr(Kf if t_ == "K" else Vf, r) for m, r in rec[t_].items()}
+                                                   for t_ in rec}}
+    out["dual_vs_shared_db"] = {"K": out["snr_db"]["K"]["plain"] - out["snr_db"]["K"]["plain_shared"],
+                                "V": out["snr_db"]["V"]["plain"] - out["snr_db"]["V"]["plain_shared"]}
+    Kh, Vh = Kf.reshape(H, N, d), Vf.reshape(H, N, d)
+    s_exact = torch.einsum("hqd,hkd->hqk", Q, Kh) / np.sqrt(d)
+    o_exact = torch.softmax(s_exact, -1) @ Vh
+    errs = {}
+    for kname, vname in (("qjl", "plain"), ("sign_mean", "sign_mean"), ("b-1+1", "plain"), ("plain", "plain")):
+        s_a = torch.einsum("hqd,hkd->hqk", Q, rec["K"][kname].reshape(H, N, d)) / np.sqrt(d)
+        ds = s_a - s_exact
+        o_a = torch.softmax(s_a, -1) @ rec["V"][vname].reshape(H, N, d)
+        cos = torch.nn.functional.cosine_similarity(o_a, o_exact, dim=-1)
+        errs[f"K {kname} / V {vname}"] = {"score_err_rel_rms": float(ds.pow(2).mean().sqrt() / s_exact.pow(2).mean().sqrt()),
+                                          "score_err_mean": float(ds.mean()), "out_cos_mean": float(cos.mean()),
+                                          "out_cos_min": float(cos.min())}
+        del s_a, ds, o_a
+    out["attention_vs_fp32"] = errs
+    from_bytes = lambda kb, vb: L * H * N * (kb + vb)
+    fp32 = L * H * N * 2 * d * 4
+    kq = d * 3 // 8 + (d + 31) // 32 * 4 + 8
+    layouts = {"configs (K codes+QJL signs+2 norms, V codes+norm)": (kq, d * 3 // 8 + 4),
+               "TurboESM sign+e_bar (K and V codes+signs+norm)": (d * 3 // 8 + d // 8 + 4, d * 3 // 8 + d // 8 + 4),
+               "TurboQuant (b-1)+1 at b=3 (K 2-bit+QJL, V 3-bit)": (d * 2 // 8 + (d + 31) // 32 * 4 + 8, d * 3 // 8 + 4)}
+    out["layouts"] = {k: {"bytes_per_token_head": kb + vb, "MiB": from_bytes(kb, vb) / 2 ** 20,
+                          "ratio_vs_fp32": fp32 / from_bytes(kb, vb)} for k, (kb, vb) in layouts.items()}
+    out["fp32_MiB"] = fp32 / 2 ** 20
+    out["layer"] = layer
+    return out
 
 
 def run_c2(args, world, rank, tq):
     dev = torch.device("cuda", torch.cuda.current_device())
-    data, PiK_h, PiV_h, (ck, tk), (cv, tv) = esm_setup(tq, replica_seed(rank), dev)
+    data, PiK_h, PiV_h, (ck, tk), (cv, tv), calib_u = esm_setup(tq, replica_seed(rank), dev)
     L, H, N, d = data.K.shape
     n = L * H * N
     lay = tq.layout(d, 3, 3)
@@ -718,6 +813,7 @@ def run_c2(args, world, rank, tq):
         res["roofline"], res["roofline_quantize"], res["roofline_quantize_value"] = att, quant, quant_v
     else:
         res["roofline"], res["roofline_attention"], res["roofline_quantize_value"] = quant, att, quant_v
+    res["variants"] = variants_c2(tq, data, PiK_h, PiV_h, ((ck, tk), (cv, tv)), calib_u, dev)
     e2e = None
     if not args.no_e2e:
         hK = K.cpu().pin_memory()

@@ -298,6 +298,46 @@ tq_status tq_dequantize(const tq_layout* layout, int32_t is_key, int64_t n_vecto
                         void* out, tq_dtype out_dtype, int64_t out_stride, void* stream);
 
 /* ------------------------------------------------------------------------
+ * tq_dequantize_sign_mean — reconstruct with TurboESM's one-bit residual
+ * correction (device).
+ *
+ * gist.science TurboESM section 2D: only the sign of each residual
+ * coordinate is stored beside the 3-bit index, and decoding adds a first-order
+ * correction with the pre-calibrated mean residual magnitude e_bar:
+ *   x_tilde = Pi^T ||x|| ( c[code] + e_bar (2*sign - 1) ).
+ * The signs are those tq_quantize_kv writes with is_key = 1 and S = the d x d
+ * identity (sign_i = (r_i >= 0), r the rotated residual); e_bar comes from
+ * tq_residual_mean. A vector then needs its codes, d sign bits and ||x||
+ * (36 bytes at d = 64, 3 bits; the rnorm plane is not read).
+ *
+ *  is_key     selects the layout's bits (key_bits or value_bits)
+ *  planes     idx, sign and norm of rows 0..n_vectors-1
+ *  e_bar      >= 0, in unit-vector coordinates
+ *  Pi, vectors_per_pi, pi_stride, out, out_dtype, out_stride as tq_dequantize
+ * Errors: TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED (n_vectors >= 2^31), TQ_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+tq_status tq_dequantize_sign_mean(const tq_layout* layout, int32_t is_key, int64_t n_vectors,
+                                  const tq_planes* planes, const float* Pi, int64_t vectors_per_pi,
+                                  int64_t pi_stride, const float* centroids, float e_bar,
+                                  void* out, tq_dtype out_dtype, int64_t out_stride, void* stream);
+
+/* ------------------------------------------------------------------------
+ * tq_residual_mean — calibrate e_bar for tq_dequantize_sign_mean (host).
+ *
+ * gist.science TurboESM section 2D ("mean residual magnitude, calibrated
+ * beforehand"): e_bar = mean over the samples u of |u - c[code(u)]|, with
+ * code(u) = #{j : u > boundaries[j]}. The samples are coordinates of rotated
+ * unit vectors, e.g. from tq_rotate_normalize on calibration data.
+ *
+ *  samples   host float [n_samples]
+ *  centroids, boundaries   host float, 2^bits and 2^bits - 1 entries
+ *  e_bar     host out
+ * Errors: TQ_ERR_INVALID_ARG.
+ * ---------------------------------------------------------------------- */
+tq_status tq_residual_mean(const float* samples, int64_t n_samples, const float* centroids,
+                           const float* boundaries, int32_t bits, double* e_bar);
+
+/* ------------------------------------------------------------------------
  * tq_search_topk — k best corpus vectors per query by estimated inner product.
  *
  * sudonull.com "TurboQuant: compresión 6x de LLM KV-cache" and news.hada.io's

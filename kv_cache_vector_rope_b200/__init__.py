@@ -67,6 +67,9 @@ _SIGNATURES = {
                                                    ctypes.c_int, _P, _P, _P]),
     "tq_dequantize": (ctypes.c_int, [ctypes.POINTER(Layout), _I32, _I64, ctypes.POINTER(_Planes), _P, _I64, _I64,
                                      _P, _P, _P, ctypes.c_int, _I64, _P]),
+    "tq_dequantize_sign_mean": (ctypes.c_int, [ctypes.POINTER(Layout), _I32, _I64, ctypes.POINTER(_Planes), _P, _I64,
+                                               _I64, _P, _F32, _P, ctypes.c_int, _I64, _P]),
+    "tq_residual_mean": (ctypes.c_int, [_P, _I64, _P, _P, _I32, ctypes.POINTER(ctypes.c_double)]),
     "tq_search_topk": (ctypes.c_int, [ctypes.POINTER(Layout), _P, ctypes.c_int, _I32, ctypes.POINTER(_Planes), _I64,
                                       _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "tq_search_workspace_bytes": (_SZ, [ctypes.POINTER(Layout), _I32, _I64, _I32]),
@@ -282,6 +285,28 @@ def tq_dequantize(lay: Layout, is_key: bool, planes: Planes, n_vectors: int, Pi:
     _check(_lib.tq_dequantize(ctypes.byref(lay), int(is_key), n_vectors, ctypes.byref(planes.c()),
                               _dev(Pi, "Pi"), vectors_per_pi, pi_stride, _ptr(S), _dev(centroids, "centroids"),
                               _dev(out, "out"), _dtype_code(out), out.stride(0), _stream(stream)))
+
+
+def tq_dequantize_sign_mean(lay: Layout, is_key: bool, planes: Planes, n_vectors: int, Pi: torch.Tensor,
+                            centroids: torch.Tensor, e_bar: float, out: torch.Tensor, vectors_per_pi: int = 1,
+                            pi_stride: int = 0, stream=None) -> None:
+    """x_tilde = Pi^T ||x|| (c[code] + e_bar (2 sign - 1)) for rows 0..n_vectors-1."""
+    if out.dim() != 2 or out.stride(1) != 1:
+        raise ValueError("out must be [n, d] with unit stride along d")
+    _check(_lib.tq_dequantize_sign_mean(ctypes.byref(lay), int(is_key), n_vectors, ctypes.byref(planes.c()),
+                                        _dev(Pi, "Pi"), vectors_per_pi, pi_stride, _dev(centroids, "centroids"),
+                                        float(e_bar), _dev(out, "out"), _dtype_code(out), out.stride(0),
+                                        _stream(stream)))
+
+
+def tq_residual_mean(samples, centroids, boundaries, bits: int) -> float:
+    """Mean |u - c[code(u)]| over host samples u (the e_bar of tq_dequantize_sign_mean)."""
+    u = np.ascontiguousarray(np.asarray(samples, dtype=np.float32).ravel())
+    c = np.ascontiguousarray(np.asarray(centroids, dtype=np.float32))
+    t = np.ascontiguousarray(np.asarray(boundaries, dtype=np.float32))
+    e = ctypes.c_double(0.0)
+    _check(_lib.tq_residual_mean(u.ctypes.data, u.size, c.ctypes.data, t.ctypes.data, bits, ctypes.byref(e)))
+    return float(e.value)
 
 
 def tq_search_workspace_bytes(lay: Layout, n_queries: int, n_db: int, k: int) -> int:

@@ -6,6 +6,10 @@
 // (K_tilde = K_hat + K_tilde_QJL). S acts on the rotated residual here, so the
 // correction is added before the single Pi^T.
 //
+// gist.science "TurboESM ..." section 2D (tq_dequantize_sign_mean): the sign
+// of each rotated residual coordinate and a calibrated mean magnitude e_bar
+// give the first-order correction x_tilde = x_hat + ||x|| e_bar (2 sign - 1).
+//
 // One CTA of d threads per vector: thread i forms rotated coordinate i, then
 // thread j forms output coordinate j = sum_i Pi[i][j] rot[i].
 #include <cuda_bf16.h>
@@ -33,6 +37,8 @@ struct DequantArgs {
   void* out;
   int out_dtype;
   int64_t out_stride;
+  int sign_mean;        // 1: TurboESM correction with e_bar (no S, no rnorm)
+  float e_bar;
 };
 
 __global__ void dequant_kernel(DequantArgs a) {
@@ -46,11 +52,16 @@ __global__ void dequant_kernel(DequantArgs a) {
   const uint8_t* row = a.idx + v * rb;
   const float nrm = a.norm[v];
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    rot[i] = nrm * __ldg(a.cent + get_code(row, i, a.bits));
-    if (a.is_key) pm[i] = ((a.sign[v * sw + (i >> 5)] >> (i & 31)) & 1u) ? 1.f : -1.f;
+    if (a.sign_mean) {
+      const float s = ((a.sign[v * sw + (i >> 5)] >> (i & 31)) & 1u) ? a.e_bar : -a.e_bar;
+      rot[i] = nrm * (__ldg(a.cent + get_code(row, i, a.bits)) + s);
+    } else {
+      rot[i] = nrm * __ldg(a.cent + get_code(row, i, a.bits));
+      if (a.is_key) pm[i] = ((a.sign[v * sw + (i >> 5)] >> (i & 31)) & 1u) ? 1.f : -1.f;
+    }
   }
   __syncthreads();
-  if (a.is_key) {
+  if (a.is_key && !a.sign_mean) {
     const float scale = static_cast<float>(kSqrtHalfPi / d) * a.rnorm[v];
     float corr[2] = {0.f, 0.f};
     for (int c = 0; c < 2; ++c) {
@@ -103,10 +114,39 @@ extern "C" tq_status tq_dequantize(const tq_layout* layout, int32_t is_key, int6
     return fail(TQ_ERR_INVALID_ARG, "pi_stride < 0 or vectors_per_pi < 1");
   DequantArgs a{d, is_key ? layout->key_bits : layout->value_bits, is_key ? 1 : 0, n_vectors, planes->idx,
                 planes->sign, planes->norm, planes->rnorm, Pi, vectors_per_pi, pi_stride, S, centroids, out,
-                out_dtype == TQ_F32 ? 0 : 1, out_stride};
+                out_dtype == TQ_F32 ? 0 : 1, out_stride, 0, 0.f};
   dequant_kernel<<<static_cast<unsigned>(n_vectors), 128, 2 * d * sizeof(float), static_cast<cudaStream_t>(stream)>>>(a);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_dequantize launch: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_dequantize_sign_mean(const tq_layout* layout, int32_t is_key, int64_t n_vectors,
+                                             const tq_planes* planes, const float* Pi, int64_t vectors_per_pi,
+                                             int64_t pi_stride, const float* centroids, float e_bar, void* out,
+                                             tq_dtype out_dtype, int64_t out_stride, void* stream) {
+  using namespace tq;
+  clear_error();
+  tq_status st = check_layout(layout);
+  if (st != TQ_OK) return st;
+  const int d = layout->d;
+  if (n_vectors < 0) return fail(TQ_ERR_INVALID_ARG, "n_vectors < 0");
+  if (n_vectors == 0) return TQ_OK;
+  if (n_vectors > 0x7fffffffLL) return fail(TQ_ERR_UNSUPPORTED, "n_vectors above 2^31-1 per call");
+  if (!planes || !planes->idx || !planes->sign || !planes->norm || !Pi || !centroids || !out)
+    return fail(TQ_ERR_INVALID_ARG, "NULL pointer argument (idx, sign and norm planes are required)");
+  if (!(e_bar >= 0.f)) return fail(TQ_ERR_INVALID_ARG, "e_bar must be >= 0");
+  if (out_dtype != TQ_F32 && out_dtype != TQ_BF16) return fail(TQ_ERR_INVALID_ARG, "out_dtype must be TQ_F32 or TQ_BF16");
+  if (out_stride < d) return fail(TQ_ERR_INVALID_ARG, "out_stride < d");
+  if (pi_stride < 0 || (pi_stride > 0 && vectors_per_pi < 1))
+    return fail(TQ_ERR_INVALID_ARG, "pi_stride < 0 or vectors_per_pi < 1");
+  DequantArgs a{d, is_key ? layout->key_bits : layout->value_bits, is_key ? 1 : 0, n_vectors, planes->idx,
+                planes->sign, planes->norm, nullptr, Pi, vectors_per_pi, pi_stride, nullptr, centroids, out,
+                out_dtype == TQ_F32 ? 0 : 1, out_stride, 1, e_bar};
+  dequant_kernel<<<static_cast<unsigned>(n_vectors), 128, 2 * d * sizeof(float), static_cast<cudaStream_t>(stream)>>>(a);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_dequantize_sign_mean launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }

@@ -303,4 +303,26 @@ tq_status tq_make_codebook(int32_t d, int32_t bits, int32_t mode, const float* s
   return TQ_OK;
 }
 
+tq_status tq_residual_mean(const float* samples, int64_t n_samples, const float* centroids, const float* boundaries,
+                           int32_t bits, double* e_bar) {
+  tq::clear_error();
+  if (bits < 1 || bits > 8) return tq::fail(TQ_ERR_INVALID_ARG, "bits must be in 1..8 (got %d)", bits);
+  if (!samples || n_samples < 1 || !centroids || !boundaries || !e_bar)
+    return tq::fail(TQ_ERR_INVALID_ARG, "NULL pointer or no samples");
+  const int nb = (1 << bits) - 1;
+  for (int j = 1; j < nb; ++j)
+    if (!(boundaries[j] > boundaries[j - 1])) return tq::fail(TQ_ERR_INVALID_ARG, "boundaries not strictly increasing");
+  double s = 0.0;
+  for (int64_t i = 0; i < n_samples; ++i) {
+    const double u = samples[i];
+    // code = #{j : u > t_j} (ties go to the lower code, as in the quantiser)
+    const int code = static_cast<int>(std::lower_bound(boundaries, boundaries + nb, static_cast<float>(u),
+                                                       [](float t, float x) { return t < x; }) -
+                                      boundaries);
+    s += std::fabs(u - static_cast<double>(centroids[code]));
+  }
+  *e_bar = s / static_cast<double>(n_samples);
+  return TQ_OK;
+}
+
 }  // extern "C"

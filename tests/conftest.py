@@ -38,4 +38,5 @@ def pytest_terminal_summary(terminalreporter):
     if L["checks"]:
         terminalreporter.write_line(
             "literal-bound ratios (worst over all checks): score err / (1e-4 |s|) where |s| >= typical scale "
-            f"{L['score_rel']:.3g}; over all scores {L['score_rel_all']:.3g}; max |out err| / 2e-3 {L['out_abs']:.3g}")
+            f"{L['score_rel']:.3g}; over all scores {L['score_rel_all']:.3g}; fp32 outputs max |err| / 2e-3 "
+            f"{L['out_abs_f32']:.3g}; bf16 outputs max |err| / (2e-3 + half spacing) {L['out_bf16_vs_rounding']:.3g}")

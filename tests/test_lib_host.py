@@ -215,3 +215,19 @@ def test_calibration_argument_errors():
         tq.tq_fit_rotation(np.zeros((0, 64), np.float32), np.eye(64, dtype=np.float32))
     with pytest.raises(tq.TQError):
         tq.tq_fit_rotation(np.full((4, 64), np.nan, np.float32), np.eye(64, dtype=np.float32))
+
+
+def test_residual_mean_matches_oracle_and_validates():
+    from oracle import sign_mean as osm
+    b = ocb.lloyd_max_beta(64, 3)
+    c = b.centroids.astype(np.float32)
+    t = (0.5 * (b.centroids[1:] + b.centroids[:-1])).astype(np.float32)
+    u = (np.random.default_rng(8).standard_normal(50000) / 8).astype(np.float32)
+    u[:7] = t[:7]                                        # ties take the lower code on both sides
+    e = tq.tq_residual_mean(u, c, t, 3)
+    ref = osm.residual_mean_magnitude(u.astype(np.float64), c.astype(np.float64), t.astype(np.float64))
+    assert abs(e - ref) <= 1e-12 * ref
+    with pytest.raises(tq.TQError):
+        tq.tq_residual_mean(u, c, t[::-1].copy(), 3)     # boundaries must increase
+    with pytest.raises(tq.TQError):
+        tq.tq_residual_mean(u[:0], c, t, 3)
