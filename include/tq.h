@@ -262,7 +262,10 @@ size_t tq_decode_workspace_bytes(const tq_layout* layout, int32_t batch, int32_t
  * no cudaMalloc/cudaFree and no allocating routine.
  *  - The first call on each device looks the array's device address up
  *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *    before any stream capture. The address is cached per device ordinal and
+ *    belongs to the device's primary context (the runtime API's): callers
+ *    that drive the device through their own driver-API contexts must make
+ *    the primary context current for these calls.
  *  - All calls share the one array and leave their data in it. Nothing needs
  *    clearing between calls, but calls that overlap on the GPU (other streams
  *    or host threads) race on it: serialise them.
