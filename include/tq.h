@@ -356,14 +356,38 @@ tq_status tq_residual_mean(const float* samples, int64_t n_samples, const float*
  *  centroids   device float, 2^key_bits entries
  *  k           1..32 (and <= n_db)
  *  top_idx     device int64 [n_queries][k], top_scores device float [n_queries][k]
- *  workspace   device scratch of tq_search_workspace_bytes() (256-B aligned)
+ *              (ids are row numbers of `db`; pass db rows [a, b) of a larger
+ *              corpus and merge with tq_search_merge_topk, offset a)
+ *  workspace   device scratch, 256-B aligned; queries run in blocks of as
+ *              many as it holds (tq_search_workspace_bytes reports the size of
+ *              one pass of up to 16,384 queries; any size from one query's
+ *              share up works, a smaller one takes more passes)
+ * Errors: TQ_ERR_INVALID_ARG, TQ_ERR_WORKSPACE (smaller than one query's
+ * share), TQ_ERR_UNSUPPORTED (d not 64, 128 or 200), TQ_ERR_CUDA.
  * ---------------------------------------------------------------------- */
 tq_status tq_search_topk(const tq_layout* layout, const void* q, tq_dtype q_dtype, int32_t n_queries,
                          const tq_planes* db, int64_t n_db, const float* Pi, const float* S,
                          const float* centroids, int32_t k, int64_t* top_idx, float* top_scores,
                          void* workspace, size_t workspace_bytes, void* stream);
 
-/* Scratch bytes tq_search_topk needs (0 on invalid arguments). */
+/* ------------------------------------------------------------------------
+ * tq_search_merge_topk — merge two per-query top-k lists (device), for a
+ * corpus searched in shards (row ranges, several calls or several GPUs).
+ *
+ * Same ranking as tq_search_topk (decreasing score, equal scores by
+ * increasing id). List X's ids are shifted by offset_x (the first corpus row
+ * of its shard); id -1 marks an empty slot and never enters. Both inputs are
+ * [n_queries][k], sorted as tq_search_topk writes them; the output, also
+ * [n_queries][k], may alias either input.
+ * Errors: TQ_ERR_INVALID_ARG (k outside 1..32, NULL, negative offsets), TQ_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+tq_status tq_search_merge_topk(int32_t n_queries, int32_t k,
+                               const int64_t* idx_a, const float* scores_a, int64_t offset_a,
+                               const int64_t* idx_b, const float* scores_b, int64_t offset_b,
+                               int64_t* idx_out, float* scores_out, void* stream);
+
+/* Scratch bytes tq_search_topk needs for one pass over min(n_queries, 16384)
+ * queries (0 on invalid arguments). */
 size_t tq_search_workspace_bytes(const tq_layout* layout, int32_t n_queries, int64_t n_db, int32_t k);
 
 /* ------------------------------------------------------------------------

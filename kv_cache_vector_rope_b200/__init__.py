@@ -72,6 +72,7 @@ _SIGNATURES = {
     "tq_residual_mean": (ctypes.c_int, [_P, _I64, _P, _P, _I32, ctypes.POINTER(ctypes.c_double)]),
     "tq_search_topk": (ctypes.c_int, [ctypes.POINTER(Layout), _P, ctypes.c_int, _I32, ctypes.POINTER(_Planes), _I64,
                                       _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
+    "tq_search_merge_topk": (ctypes.c_int, [_I32, _I32, _P, _P, _I64, _P, _P, _I64, _P, _P, _P]),
     "tq_search_workspace_bytes": (_SZ, [ctypes.POINTER(Layout), _I32, _I64, _I32]),
     "tq_fit_rotation": (ctypes.c_int, [_I32, _P, _I64, _P, _P]),
     "tq_rotate_normalize": (ctypes.c_int, [_I32, _P, _I64, _P, _P, ctypes.POINTER(_I64)]),
@@ -323,6 +324,16 @@ def tq_search_topk(lay: Layout, q: torch.Tensor, db: Planes, n_db: int, Pi: torc
                                n_db, _dev(Pi, "Pi"), _dev(S, "S"), _dev(centroids, "centroids"), k,
                                _dev(top_idx, "top_idx"), _dev(top_scores, "top_scores"), _dev(workspace, "workspace"),
                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def tq_search_merge_topk(idx_a: torch.Tensor, scores_a: torch.Tensor, offset_a: int, idx_b: torch.Tensor,
+                         scores_b: torch.Tensor, offset_b: int, idx_out: torch.Tensor, scores_out: torch.Tensor,
+                         stream=None) -> None:
+    """Merges two [n_queries, k] top-k lists (ids shifted by their shard offsets) into idx_out / scores_out."""
+    nq, k = idx_a.shape
+    _check(_lib.tq_search_merge_topk(nq, k, _dev(idx_a, "idx_a"), _dev(scores_a, "scores_a"), offset_a,
+                                     _dev(idx_b, "idx_b"), _dev(scores_b, "scores_b"), offset_b,
+                                     _dev(idx_out, "idx_out"), _dev(scores_out, "scores_out"), _stream(stream)))
 
 
 def tq_fit_rotation(X, Pi_rand) -> np.ndarray:

@@ -31,6 +31,7 @@ constexpr int kSThreads = 256;
 constexpr int kSRows = 8;          // queries per CTA
 constexpr int kChunk = 8192;       // corpus vectors per CTA
 constexpr int kMaxK = 32;
+constexpr int kServeBlock = 16384;  // queries per pass with the workspace tq_search_workspace_bytes reports
 
 struct SearchArgs {
   int d, bits, nq, k;
@@ -247,6 +248,35 @@ __global__ void search_merge(SearchArgs a) {
   }
 }
 
+// Merge of two per-query top-k lists (one warp per query): list A enters as
+// is, B's entries are inserted; ids are shifted by each list's offset, and -1
+// (an empty slot) never enters. Inputs are read before any output is written,
+// so the output may alias either input.
+__global__ void search_merge_lists(int nq, int k, const int64_t* ia, const float* sa, int64_t oa, const int64_t* ib,
+                                   const float* sb, int64_t ob, int64_t* io, float* so) {
+  const int lane = threadIdx.x & 31;
+  const int64_t q = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (q >= nq) return;
+  const int64_t base = q * k;
+  const int64_t a_i = lane < k ? ia[base + lane] : -1;
+  const float a_s = lane < k ? sa[base + lane] : -INFINITY;
+  const int64_t b_i = lane < k ? ib[base + lane] : -1;
+  const float b_s = lane < k ? sb[base + lane] : -INFINITY;
+  float ms = a_i >= 0 ? a_s : -INFINITY;
+  int64_t mi = a_i >= 0 ? a_i + oa : INT64_MAX;
+  const int64_t gb = b_i >= 0 ? b_i + ob : INT64_MAX;
+  unsigned m = __ballot_sync(0xffffffffu, b_i >= 0);
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    list_insert(ms, mi, k, __shfl_sync(0xffffffffu, b_s, src), __shfl_sync(0xffffffffu, gb, src));
+  }
+  if (lane < k) {
+    io[base + lane] = mi == INT64_MAX ? -1 : mi;
+    so[base + lane] = ms;
+  }
+}
+
 size_t search_ws(int d, int nq, int64_t n_db, int k) {
   const int64_t chunks = (n_db + kChunk - 1) / kChunk;
   const size_t qs = ((size_t(nq) * 2 * d * 4 + 255) / 256) * 256;
@@ -260,7 +290,7 @@ size_t search_ws(int d, int nq, int64_t n_db, int k) {
 
 extern "C" size_t tq_search_workspace_bytes(const tq_layout* layout, int32_t n_queries, int64_t n_db, int32_t k) {
   if (tq::check_layout(layout) != TQ_OK || n_queries < 1 || n_db < 1 || k < 1 || k > tq::kMaxK) return 0;
-  return tq::search_ws(layout->d, n_queries, n_db, k);
+  return tq::search_ws(layout->d, n_queries < tq::kServeBlock ? n_queries : tq::kServeBlock, n_db, k);
 }
 
 extern "C" tq_status tq_search_topk(const tq_layout* layout, const void* q, tq_dtype q_dtype, int32_t n_queries,
@@ -278,70 +308,96 @@ extern "C" tq_status tq_search_topk(const tq_layout* layout, const void* q, tq_d
       !top_scores)
     return fail(TQ_ERR_INVALID_ARG, "NULL pointer argument");
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_F32 or TQ_BF16");
-  const size_t need = search_ws(d, n_queries, n_db, k);
-  if (!workspace || workspace_bytes < need)
-    return fail(TQ_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
+  // Queries run in blocks of as many as the workspace holds (one pass when it
+  // holds them all).
+  if (!workspace || workspace_bytes < search_ws(d, 1, n_db, k))
+    return fail(TQ_ERR_WORKSPACE, "workspace of at least %zu bytes needed (got %zu)", search_ws(d, 1, n_db, k),
+                workspace_bytes);
   if (!aligned(workspace, 256)) return fail(TQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  SearchArgs a{};
-  a.d = d;
-  a.bits = layout->key_bits;
-  a.nq = n_queries;
-  a.k = k;
-  a.n_db = n_db;
-  a.n_chunks = static_cast<int>((n_db + kChunk - 1) / kChunk);
-  if ((n_queries + kSRows - 1) / kSRows > 65535) return fail(TQ_ERR_UNSUPPORTED, "too many queries per call (max 524280)");
-  a.q = q;
-  a.q_dtype = q_dtype == TQ_F32 ? 0 : 1;
-  a.idx = db->idx;
-  a.sign = db->sign;
-  a.norm = db->norm;
-  a.rnorm = db->rnorm;
-  a.Pi = Pi;
-  a.S = S;
-  a.cent = centroids;
-  char* w = static_cast<char*>(workspace);
-  a.qs = reinterpret_cast<float*>(w);
-  w += ((size_t(n_queries) * 2 * d * 4 + 255) / 256) * 256;
-  a.cand_s = reinterpret_cast<float*>(w);
-  w += ((size_t(n_queries) * a.n_chunks * k * 4 + 255) / 256) * 256;
-  a.cand_i = reinterpret_cast<int64_t*>(w);
-  a.top_idx = top_idx;
-  a.top_s = top_scores;
+  int qb = n_queries < kServeBlock ? n_queries : kServeBlock;
+  while (qb > 1 && search_ws(d, qb, n_db, k) > workspace_bytes) qb = (qb + 1) / 2;
+  while (qb < n_queries && search_ws(d, qb + 1, n_db, k) <= workspace_bytes && qb < kServeBlock) ++qb;
+  const int n_chunks = static_cast<int>((n_db + kChunk - 1) / kChunk);
+  if (d != 64 && d != 128 && d != 200) return fail(TQ_ERR_UNSUPPORTED, "tq_search_topk: d=%d not built (64, 128, 200)", d);
+  const size_t elem = q_dtype == TQ_F32 ? 4 : 2;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  search_prologue<<<n_queries, 128, d * sizeof(double) + d * sizeof(float), s>>>(a);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) {
-    const int nc = 1 << a.bits;
-    const size_t smem = sizeof(float) * (d * nc * kSRows + (d / 4) * 16 * kSRows + 8 * kSRows * 32) +
-                        sizeof(int64_t) * 8 * kSRows * 32;
-    dim3 grid(a.n_chunks, (n_queries + kSRows - 1) / kSRows);
-    switch (d) {
-      case 64:
-        cudaFuncSetAttribute(search_main<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        search_main<64><<<grid, kSThreads, smem, s>>>(a);
-        count_launch();
-        break;
-      case 128:
-        cudaFuncSetAttribute(search_main<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        search_main<128><<<grid, kSThreads, smem, s>>>(a);
-        count_launch();
-        break;
-      case 200:
-        cudaFuncSetAttribute(search_main<200>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        search_main<200><<<grid, kSThreads, smem, s>>>(a);
-        count_launch();
-        break;
-      default:
-        return fail(TQ_ERR_UNSUPPORTED, "tq_search_topk: d=%d not built (64, 128, 200)", d);
-    }
-    e = cudaGetLastError();
-  }
-  if (e == cudaSuccess) {
-    search_merge<<<(n_queries + 3) / 4, 128, 0, s>>>(a);
+  cudaError_t e = cudaSuccess;
+  for (int q0 = 0; q0 < n_queries && e == cudaSuccess; q0 += qb) {
+    const int nb = n_queries - q0 < qb ? n_queries - q0 : qb;
+    SearchArgs a{};
+    a.d = d;
+    a.bits = layout->key_bits;
+    a.nq = nb;
+    a.k = k;
+    a.n_db = n_db;
+    a.n_chunks = n_chunks;
+    a.q = static_cast<const char*>(q) + size_t(q0) * d * elem;
+    a.q_dtype = q_dtype == TQ_F32 ? 0 : 1;
+    a.idx = db->idx;
+    a.sign = db->sign;
+    a.norm = db->norm;
+    a.rnorm = db->rnorm;
+    a.Pi = Pi;
+    a.S = S;
+    a.cent = centroids;
+    char* w = static_cast<char*>(workspace);
+    a.qs = reinterpret_cast<float*>(w);
+    w += ((size_t(nb) * 2 * d * 4 + 255) / 256) * 256;
+    a.cand_s = reinterpret_cast<float*>(w);
+    w += ((size_t(nb) * n_chunks * k * 4 + 255) / 256) * 256;
+    a.cand_i = reinterpret_cast<int64_t*>(w);
+    a.top_idx = top_idx + int64_t(q0) * k;
+    a.top_s = top_scores + int64_t(q0) * k;
+    search_prologue<<<nb, 128, d * sizeof(double) + d * sizeof(float), s>>>(a);
     count_launch();
     e = cudaGetLastError();
+    if (e == cudaSuccess) {
+      const int nc = 1 << a.bits;
+      const size_t smem = sizeof(float) * (d * nc * kSRows + (d / 4) * 16 * kSRows + 8 * kSRows * 32) +
+                          sizeof(int64_t) * 8 * kSRows * 32;
+      dim3 grid(n_chunks, (nb + kSRows - 1) / kSRows);
+      switch (d) {
+        case 64:
+          cudaFuncSetAttribute(search_main<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+          search_main<64><<<grid, kSThreads, smem, s>>>(a);
+          break;
+        case 128:
+          cudaFuncSetAttribute(search_main<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+          search_main<128><<<grid, kSThreads, smem, s>>>(a);
+          break;
+        default:
+          cudaFuncSetAttribute(search_main<200>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+          search_main<200><<<grid, kSThreads, smem, s>>>(a);
+          break;
+      }
+      count_launch();
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+      search_merge<<<(nb + 3) / 4, 128, 0, s>>>(a);
+      count_launch();
+      e = cudaGetLastError();
+    }
   }
   if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_search_topk launch: %s", cudaGetErrorString(e));
+  return TQ_OK;
+}
+
+extern "C" tq_status tq_search_merge_topk(int32_t n_queries, int32_t k, const int64_t* idx_a, const float* scores_a,
+                                         int64_t offset_a, const int64_t* idx_b, const float* scores_b,
+                                         int64_t offset_b, int64_t* idx_out, float* scores_out, void* stream) {
+  using namespace tq;
+  clear_error();
+  if (n_queries < 0) return fail(TQ_ERR_INVALID_ARG, "n_queries < 0");
+  if (n_queries == 0) return TQ_OK;
+  if (k < 1 || k > kMaxK) return fail(TQ_ERR_INVALID_ARG, "k must be in [1, 32] (got %d)", k);
+  if (!idx_a || !scores_a || !idx_b || !scores_b || !idx_out || !scores_out)
+    return fail(TQ_ERR_INVALID_ARG, "NULL pointer argument");
+  if (offset_a < 0 || offset_b < 0) return fail(TQ_ERR_INVALID_ARG, "offsets must be >= 0");
+  search_merge_lists<<<(n_queries + 3) / 4, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      n_queries, k, idx_a, scores_a, offset_a, idx_b, scores_b, offset_b, idx_out, scores_out);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_search_merge_topk launch: %s", cudaGetErrorString(e));
   return TQ_OK;
 }

@@ -231,3 +231,18 @@ def test_residual_mean_matches_oracle_and_validates():
         tq.tq_residual_mean(u, c, t[::-1].copy(), 3)     # boundaries must increase
     with pytest.raises(tq.TQError):
         tq.tq_residual_mean(u[:0], c, t, 3)
+
+
+def test_search_merge_host_validation():
+    f = tq._lib.tq_search_merge_topk
+    p = 0x1000
+    assert f(0, 10, p, p, 0, p, p, 0, p, p, None) == tq.TQ_OK              # nothing to merge
+    assert f(4, 33, p, p, 0, p, p, 0, p, p, None) == tq.TQ_ERR_INVALID_ARG  # k above 32
+    assert f(4, 0, p, p, 0, p, p, 0, p, p, None) == tq.TQ_ERR_INVALID_ARG
+    assert f(4, 10, p, p, -1, p, p, 0, p, p, None) == tq.TQ_ERR_INVALID_ARG
+    assert f(4, 10, 0, p, 0, p, p, 0, p, p, None) == tq.TQ_ERR_INVALID_ARG
+    lay = tq.layout(128, 3, 3)
+    one = tq._lib.tq_search_workspace_bytes(ctypes.byref(lay), 1, 100000, 10)
+    many = tq._lib.tq_search_workspace_bytes(ctypes.byref(lay), 100000, 100000, 10)
+    cap = tq._lib.tq_search_workspace_bytes(ctypes.byref(lay), 16384, 100000, 10)
+    assert 0 < one < cap == many                       # one pass holds at most 16,384 queries
