@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
   TQ_OK = 0,
   TQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or combination   */
-  TQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement   */
+  TQ_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement  */
   TQ_ERR_CUDA = 3,          /* a CUDA runtime call failed (see error string)  */
   TQ_ERR_WORKSPACE = 4      /* workspace missing or smaller than required    */
 } tq_status;

@@ -16,6 +16,10 @@
 //                sign bits; V is accumulated in rotated coordinates with an
 //                online softmax; each CTA leaves (m, l, acc) for its split.
 //   3. combine   merges the splits and applies Pi_V^T once per query row.
+// Shapes the fused tensor-core kernel takes (d = 128, four query heads per KV
+// head, one query each, 3-bit values; tq_decode_tc.cu) go there instead;
+// TQ_DECODE_PATH=v1 or v2 keeps them on these kernels (v2: the table kernel of
+// tq_decode_v2.cuh, v1: the general one).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
