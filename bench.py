@@ -968,15 +968,65 @@ def run_incremental_c3(args, tq, lay, Q, kp, vp, out, ws, Pi, S, cd, td, status,
         marks[i][2].record()
     torch.cuda.synchronize()
     launches = tq.tq_kernel_launches() - n0
-    barrier(world)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
     per_token = max_over_ranks(world, statistics.mean(m[0].elapsed_time(m[2]) for m in marks))
     append_l0 = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+
+    # The same steps, each captured once as a CUDA graph (the host's launch
+    # cost leaves the timed region), replayed in order.
+    def one_step(i, sl):
+        for l in range(L):
+            tq.tq_append_kv(lay, True, kn[i, l], kp[l], N, sl, Pi, cd, td, S=S, positions=kpos[i], rope_base=base,
+                            d_status=status)
+            tq.tq_append_kv(lay, False, vn[i, l], vp[l], N, sl, Pi, cd, td, d_status=status)
+            tq.tq_decode_attention(lay, Q[l], kp[l], vp[l], HKV, sl + 1, Pi, Pi, S, cd, cd, out[l], ws,
+                                   q_positions=qpos[i], rope_base=base, ctx_stride=N, d_status=status)
+
+    graph = {}
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        graphs = []
+        with torch.cuda.stream(side):
+            for i, sl in enumerate(slots):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    one_step(i, sl)
+                graphs.append(g)
+            ga = torch.cuda.CUDAGraph()                # 100 appends of one layer's 64 keys
+            with torch.cuda.graph(ga, stream=side):
+                for _ in range(100):
+                    tq.tq_append_kv(lay, True, kn[0, 0], kp[0], N, slots[0], Pi, cd, td, S=S, positions=kpos[0],
+                                    rope_base=base, d_status=status)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        barrier(world)
+        s0, s1 = ev(), ev()
+        s0.record()
+        for g in graphs:
+            g.replay()
+        s1.record()
+        torch.cuda.synchronize()
+        a0, a1 = ev(), ev()
+        a0.record()
+        ga.replay()
+        a1.record()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, f"device status {int(status.item())}"
+        g_tok = max_over_ranks(world, s0.elapsed_time(s1) / T)
+        graph = {"us_per_generated_token": 1e3 * g_tok, "tokens_per_s": world * B / (g_tok * 1e-3),
+                 "append_call_us": 1e3 * a0.elapsed_time(a1) / 100}
+        del graphs, ga
+    except Exception as exc:  # capture is reported, not required
+        graph = {"error": str(exc).splitlines()[0][:200]}
+    barrier(world)
     return {"us_per_generated_token": 1e3 * per_token, "tokens_per_s": world * B / (per_token * 1e-3),
             "layers": L, "steps": T, "append_us_layer0": 1e3 * append_l0, "gpu_launches": launches,
+            "graph": graph,
             "note": (f"per step and layer: tq_append_kv of {streams} keys (RoPE) and {streams} values at slot "
-                     f"N-{T}+i, then tq_decode_attention over slot+1 tokens (ctx_stride {N}); "
-                     f"tokens_per_s counts the batch's {B} sequences")}
+                     f"N-{T}+i, then tq_decode_attention over slot+1 tokens (ctx_stride {N}); eager launches from "
+                     f"Python, and each step replayed from a CUDA graph; tokens_per_s counts the batch's {B} "
+                     f"sequences")}
 
 
 def run_e2e_c3(args, tq, lay, K, V, Q, kp, vp, out, ws, Pi, S, cd, td, status, shape, world):

@@ -143,7 +143,8 @@ tq_status tq_make_codebook(int32_t d, int32_t bits, int32_t mode,
  *   keys: r = y - ||x'|| centroids[code];  sign_i = ((S r)_i >= 0)
  * Codes and signs equal those of exact arithmetic: any coordinate (or sign)
  * whose fp32 margin is within a guard band of its decision is recomputed in
- * fp64 before it is stored.
+ * fp64 before it is stored. Calls of at most 1024 vectors with one shared Pi
+ * run entirely in fp64, one CTA per vector (the kernel of tq_append_kv).
  *
  *  layout          d and the bits of this tensor (key_bits if is_key, else
  *                  value_bits)

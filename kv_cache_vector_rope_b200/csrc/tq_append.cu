@@ -69,10 +69,33 @@ __device__ __forceinline__ double block_sum(double v, double* red) {
   return t;
 }
 
+// M (row-major D x D, 16-byte aligned) into shared memory at the padded
+// stride, float4 loads issued eight at a time so that the L2 latency is paid
+// once per eight loads rather than once per load.
 template <int D>
 __device__ __forceinline__ void stage_matrix(float* M, const float* __restrict__ src) {
   constexpr int T = threads_for(D);
-  for (int e = threadIdx.x; e < D * D; e += T) M[(e / D) * AppendSmem<D>::kLd + e % D] = __ldg(src + e);
+  constexpr int kV = D * D / 4;                      // float4 in the matrix
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  for (int base = 0; base < kV; base += 8 * T) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = base + u * T + threadIdx.x;
+      if (e < kV) v[u] = __ldg(s4 + e);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = base + u * T + threadIdx.x;
+      if (e < kV) {
+        float* dst = M + ((4 * e) / D) * AppendSmem<D>::kLd + (4 * e) % D;   // D % 4 == 0: a row holds whole float4s
+        dst[0] = v[u].x;
+        dst[1] = v[u].y;
+        dst[2] = v[u].z;
+        dst[3] = v[u].w;
+      }
+    }
+  }
 }
 
 template <int D>
@@ -170,6 +193,21 @@ cudaError_t launch_append(const AppendArgs& a, int64_t n, cudaStream_t st) {
 }
 
 }  // namespace
+
+// Small quantise calls (tq_quantize_kv with a shared Pi and few vectors) run
+// on the same exact kernel: vector v to plane row v.
+cudaError_t append_quantize(int d, int bits, bool is_key, const void* x, int dtype, int64_t n, int64_t row_stride,
+                            const int32_t* pos, float rope_base, const float* Pi, const float* S, const float* cent,
+                            const float* bnd, const tq_planes* out, int32_t* d_status, cudaStream_t st) {
+  AppendArgs a{x, dtype, row_stride, pos, static_cast<double>(rope_base), Pi, S, cent, bnd, bits, is_key ? 1 : 0,
+               out->idx, is_key ? out->sign : nullptr, out->norm, is_key ? out->rnorm : nullptr, 1, 0, d_status};
+  switch (d) {
+    case 64: return launch_append<64>(a, n, st);
+    case 128: return launch_append<128>(a, n, st);
+    default: return launch_append<200>(a, n, st);
+  }
+}
+
 }  // namespace tq
 
 extern "C" tq_status tq_append_kv(const tq_layout* layout, int32_t is_key, const void* x, tq_dtype x_dtype,

@@ -32,6 +32,7 @@ using namespace dev;
 
 constexpr int kThreads = 256;
 constexpr int kTV = 64;        // vectors per tile
+constexpr int64_t kExactMaxVectors = 1024;   // up to this many: the exact per-vector kernel
 constexpr int kJC = 32;        // reduction chunk of the GEMMs
 // Guard bands (relative to ||x|| for codes and to ||r|| for signs). The fp32
 // error of a d<=256 dot product here is below 3e-7 of those scales.
@@ -372,12 +373,15 @@ cudaError_t launch(const QuantArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-// TQ_QUANTIZE_PATH=cuda-core selects the CUDA-core kernel even where the
-// tensor-core one applies (both compute the same planes; tests cover both).
-bool getenv_force_cuda_core() {
+// TQ_QUANTIZE_PATH selects a kernel where several apply (all compute the
+// same planes; tests cover each): "cuda-core" the tiled CUDA-core kernel,
+// "tensor-core" the tensor-core kernel where it applies (no exact small-call
+// path), unset or anything else the default choice.
+bool getenv_path(const char* name) {
   const char* e = std::getenv("TQ_QUANTIZE_PATH");
-  return e != nullptr && std::strcmp(e, "cuda-core") == 0;
+  return e != nullptr && std::strcmp(e, name) == 0;
 }
+bool getenv_force_cuda_core() { return getenv_path("cuda-core"); }
 
 }  // namespace tq
 
@@ -408,6 +412,16 @@ extern "C" tq_status tq_quantize_kv(const tq_layout* layout, int32_t is_key, con
               out->idx, is_key ? out->sign : nullptr, out->norm, is_key ? out->rnorm : nullptr, d_status};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool rope = positions != nullptr && rope_base > 0.f;
+  // Few vectors and one shared Pi: the exact one-CTA-per-vector kernel (a
+  // tile kernel would run on a handful of SMs). TQ_QUANTIZE_PATH=cuda-core
+  // keeps such calls on the tiled CUDA-core kernel.
+  if (!getenv_force_cuda_core() && !getenv_path("tensor-core") && n_vectors <= kExactMaxVectors && pi_stride == 0 &&
+      (d == 64 || d == 128 || d == 200) && aligned(Pi, 16) && (!S || aligned(S, 16))) {
+    cudaError_t e = append_quantize(d, bits, is_key != 0, x, x_dtype == TQ_F32 ? 0 : 1, n_vectors, row_stride,
+                                    positions, rope_base, Pi, S, centroids, boundaries, out, d_status, s);
+    if (e != cudaSuccess) return fail(TQ_ERR_CUDA, "tq_quantize_kv launch: %s", cudaGetErrorString(e));
+    return TQ_OK;
+  }
   if (!getenv_force_cuda_core() && tc_quantize_supported(d, x_dtype, rope, vectors_per_pi, pi_stride, x, row_stride))
     return tc_quantize(d, is_key != 0, bits, x, n_vectors, row_stride, Pi, vectors_per_pi, pi_stride, S, centroids,
                        boundaries, out, d_status, s);

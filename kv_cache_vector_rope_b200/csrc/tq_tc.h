@@ -18,4 +18,10 @@ tq_status tc_quantize(int d, bool is_key, int bits, const void* x, int64_t n, in
                       int64_t vectors_per_pi, int64_t pi_stride, const float* S, const float* cent, const float* bnd,
                       const tq_planes* out, int32_t* d_status, cudaStream_t st);
 
+// Exact fp64 quantisation, one CTA per vector (tq_append.cu): vector v to
+// plane row v. For calls with few vectors and one shared Pi.
+cudaError_t append_quantize(int d, int bits, bool is_key, const void* x, int dtype, int64_t n, int64_t row_stride,
+                            const int32_t* pos, float rope_base, const float* Pi, const float* S, const float* cent,
+                            const float* bnd, const tq_planes* out, int32_t* d_status, cudaStream_t st);
+
 }  // namespace tq

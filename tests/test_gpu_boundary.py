@@ -1,11 +1,13 @@
-"""Both quantisers on inputs built at and beside their decision points.
+"""The quantisers on inputs built at and beside their decision points.
 
 Rows from tests/boundary.py put a rotated coordinate at t_j + delta sigma_d or
 a projected residual at delta ||r|| (delta in {0, +-1e-9, +-1e-7, +-1e-6,
 +-2e-6}), plus rows with one channel x1e4. The tensor-core quantiser (bf16
-input) and the CUDA-core quantiser (bf16 and fp32 input) must reproduce the
+input), the CUDA-core quantiser (bf16 and fp32 input) and the exact per-vector
+kernel that small calls use (bf16 input) must reproduce the
 oracle's codes and signs exactly: their guard bands send every such row to
-the fp64 fixup. The only differences allowed are where the oracle's own fp64
+the fp64 fixup; the exact per-vector kernel (small calls) decides everything in
+fp64. The only differences allowed are where the oracle's own fp64
 value is within 1e-12 (sigma_d for codes, ||r|| for signs) of the decision
 point, below the resolution two fp64 summation orders can agree on.
 """
@@ -38,7 +40,7 @@ def _dev(x):
 
 
 @pytest.mark.parametrize("d,bits", [(128, 3), (64, 3), (128, 2), (128, 4)])
-@pytest.mark.parametrize("path", ["tensor-core", "cuda-core-bf16", "cuda-core-fp32"])
+@pytest.mark.parametrize("path", ["tensor-core", "cuda-core-bf16", "cuda-core-fp32", "exact-bf16"])
 def test_quantizers_exact_at_decision_points(d, bits, path, monkeypatch):
     c, t = _book(d, bits)
     Pi = synth.random_rotation(d, 0)
@@ -47,7 +49,9 @@ def test_quantizers_exact_at_decision_points(d, bits, path, monkeypatch):
                                              c.astype(np.float64), t.astype(np.float64), seed=d + bits)
     X = np.concatenate([X, X[:37]])                   # several tiles' worth plus a ragged tail
     if path == "tensor-core":
-        monkeypatch.delenv("TQ_QUANTIZE_PATH", raising=False)
+        monkeypatch.setenv("TQ_QUANTIZE_PATH", "tensor-core")
+    elif path.startswith("exact"):
+        monkeypatch.delenv("TQ_QUANTIZE_PATH", raising=False)     # a small call: the exact per-vector kernel
     else:
         monkeypatch.setenv("TQ_QUANTIZE_PATH", "cuda-core")
     x = torch.as_tensor(X, device="cuda")

@@ -325,12 +325,13 @@ def test_tensor_core_and_cuda_core_quantize_paths(d, bits, monkeypatch):
     S = synth.gaussian_projection(d, 3)
     for is_key in (True, False):
         ref = quantize_ref(X64, d, bits, is_key, Pi, S if is_key else None)
-        monkeypatch.delenv("TQ_QUANTIZE_PATH", raising=False)
+        monkeypatch.setenv("TQ_QUANTIZE_PATH", "tensor-core")
         p_tc = quantize_gpu(Xb.cuda(), d, bits, is_key, Pi, S if is_key else None)
         monkeypatch.setenv("TQ_QUANTIZE_PATH", "cuda-core")
         p_cc = quantize_gpu(Xb.cuda(), d, bits, is_key, Pi, S if is_key else None)
         monkeypatch.delenv("TQ_QUANTIZE_PATH")
-        for p in (p_tc, p_cc):
+        p_ex = quantize_gpu(Xb.cuda(), d, bits, is_key, Pi, S if is_key else None)   # small call: exact kernel
+        for p in (p_tc, p_cc, p_ex):
             P.compare_quantized(P.host_planes(p), ref, d, bits, is_key)
 
 
