@@ -1037,7 +1037,9 @@ def run_e2e_c3(args, tq, lay, K, V, Q, kp, vp, out, ws, Pi, S, cd, td, status, s
     L = len(K)
     per_layer = 2 * K[0].numel() * K[0].element_size()
     avail = psutil.virtual_memory().available
-    pool = max(1, min(L, int(0.3 * avail // per_layer)))
+    # Pinned host copies of up to 30% of the free host memory, shared by the
+    # ranks of this node (each takes its 1/world part).
+    pool = max(1, min(L, int(0.3 / world * avail // per_layer)))
     hostK = [torch.empty_like(K[i], device="cpu").pin_memory() for i in range(pool)]
     hostV = [torch.empty_like(V[i], device="cpu").pin_memory() for i in range(pool)]
     for i in range(pool):
