@@ -77,3 +77,36 @@ def test_bench_rejects_gpus_that_differ_from_the_launcher():
                env_extra={"WORLD_SIZE": "2", "RANK": "0", "LOCAL_RANK": "0"})
     assert r.returncode != 0
     assert "WORLD_SIZE=2" in r.stderr
+
+
+@pytest.mark.parametrize("config", [2, 3, 4, 5])
+def test_reference_arm_of_every_config_runs_on_the_host(config):
+    import json
+    r = _bench(["--impl", "reference", "--config", str(config), "--steps", "1", "--warmup", "0", "--cpu-budget", "0.3"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    res = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][-1])
+    assert res["impl"] == "reference" and res["config"]["config_id"] == config
+    assert res["value"] > 0 and res["cpu_baseline"]["kind"] == "oracle"
+    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["e2e"]["value"] == res["value"]
+
+
+def test_bench_roofline_and_traffic_helpers():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.packed_bytes(128, 3, True) == 72 and bench.packed_bytes(128, 3, False) == 52
+    assert bench.packed_bytes(64, 3, True) == 40 and bench.packed_bytes(200, 3, True) == 111
+    peaks = {"hbm_gbs": 1000.0, "hbm_src": "measured"}
+    r = bench.hbm_roofline("k", 2e9, 1e-3, peaks, "unit")          # 2 GB in 1 ms = 2000 GB/s
+    assert abs(r["achieved"] - 2000.0) < 1e-9 and abs(r["frac"] - 2.0) < 1e-12 and r["traffic"] is None
+    # a traffic entry counts only while the kernel sources hash to its sha
+    key = next(iter(bench.TRAFFIC))
+    e = bench.TRAFFIC[key]
+    current = bench._sources_sha(e["sources"]) == e["sha"]
+    t = bench.traffic_for(key, 10)
+    assert (t == e["bytes_per_unit"] * 10) if current else (t is None)
+    saved = dict(e)
+    try:
+        e["sha"] = "0" * 16
+        assert bench.traffic_for(key, 10) is None
+    finally:
+        e.update(saved)
