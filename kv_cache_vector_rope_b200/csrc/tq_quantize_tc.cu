@@ -642,7 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1) quantize_tc_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 constexpr int kFixThreads = 512;       // 16 warps
 constexpr int kFixWarps = kFixThreads / 32;
-constexpr int kFixList = 8192;         // rows scanned per round (list capacity)
+constexpr int kFixList = 16384;        // rows scanned per round (list capacity; one
+                                       // round covers a CTA's share of a 2M-row call)
 constexpr int kFixBatch = 4;           // rows per warp at a time
 
 template <int D, bool KEY>
@@ -735,21 +736,27 @@ __device__ __forceinline__ void fix_batch(const TcArgs& a, const int64_t (&rows)
   constexpr int kNb = (1 << BITS) - 1;
   constexpr int G = D / 32;
   const int lane = threadIdx.x & 31;
-  // x of every row as fp64 into the scratch, and ||x||.
+  // x of every row as fp64 into the scratch, and ||x||. The loads of all rows
+  // are issued before any arithmetic; rows r >= n repeat row 0 (a valid
+  // address) and their values are not used.
   double n64[kFixBatch];
+  float xf[kFixBatch][G];
+#pragma unroll
+  for (int r = 0; r < kFixBatch; ++r) {
+    const __nv_bfloat16* xr = a.x + rows[r] * a.row_stride;
+#pragma unroll
+    for (int c = 0; c < G; ++c) xf[r][c] = __bfloat162float(xr[32 * c + lane]);
+  }
 #pragma unroll
   for (int r = 0; r < kFixBatch; ++r) {
     double nn = 0.0;
-    if (r < n) {
-      const __nv_bfloat16* xr = a.x + rows[r] * a.row_stride;
 #pragma unroll
-      for (int c = 0; c < G; ++c) {
-        const double xv = static_cast<double>(__bfloat162float(xr[32 * c + lane]));
-        scr[r * D + 32 * c + lane] = xv;
-        nn = fma(xv, xv, nn);
-      }
+    for (int c = 0; c < G; ++c) {
+      const double xv = static_cast<double>(xf[r][c]);
+      scr[r * D + 32 * c + lane] = xv;
+      nn = fma(xv, xv, nn);
     }
-    n64[r] = sqrt(warp_sum(nn));
+    n64[r] = r < n ? sqrt(warp_sum(nn)) : 0.0;
   }
   __syncwarp();
   double y[kFixBatch][G];
