@@ -91,12 +91,12 @@ WORKLOADS = {
 # kernel ends, so the write bytes are a lower bound. The quantise entries sum
 # the main kernel and its fixup (the call the roofline times).
 TRAFFIC = {
-    "decode_fused3_d128": {"bytes_per_unit": (65_943_552 + 246_272) / 524_288, "sha": "d958b2d61582ac83",
+    "decode_fused3_d128": {"bytes_per_unit": (65_936_640 + 58_624) / 524_288, "sha": "d958b2d61582ac83",
                            "sources": ["tq_decode_tc.cu", "tq_decode_tc.h", "tq_sm100.cuh"]},
-    "quantize_tc_key3_d128": {"bytes_per_unit": (134_565_376 + 13_969_152 + 2_681_088) / 524_288,
-                              "sha": "3cf723122ba79b6b", "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
-    "quantize_tc_value3_d128": {"bytes_per_unit": (134_330_880 + 9_040_640 + 2_406_656) / 524_288,
-                                "sha": "3cf723122ba79b6b",
+    "quantize_tc_key3_d128": {"bytes_per_unit": (134_523_136 + 17_896_448 + 2_691_072) / 524_288,
+                              "sha": "466b735e2112a69a", "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
+    "quantize_tc_value3_d128": {"bytes_per_unit": (134_339_072 + 9_486_336 + 2_416_640) / 524_288,
+                                "sha": "466b735e2112a69a",
                                 "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
 }
 
