@@ -645,6 +645,7 @@ constexpr int kFixWarps = kFixThreads / 32;
 constexpr int kFixList = 16384;        // rows scanned per round (list capacity; one
                                        // round covers a CTA's share of a 2M-row call)
 constexpr int kFixBatch = 4;           // rows per warp at a time
+constexpr int kFixGridRows = 8192;     // rows per fixup CTA when the call is smaller than the grid
 
 template <int D, bool KEY>
 struct FixCfg {
@@ -923,7 +924,9 @@ cudaError_t launch_tc(const TcArgs& a, const CUtensorMap& map, cudaStream_t st) 
   e = cudaFuncSetAttribute(quantize_fixup<D, KEY, BITS, PH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(fix_smem));
   if (e != cudaSuccess) return e;
-  const int64_t fix_ctas = (a.n + kFixList - 1) / kFixList;
+  // One CTA per 8,192 rows, at most one per SM (a CTA's share then fits one
+  // scan window up to 148 x 16,384 rows).
+  const int64_t fix_ctas = (a.n + kFixGridRows - 1) / kFixGridRows;
   quantize_fixup<D, KEY, BITS, PH><<<static_cast<int>(fix_ctas < sms ? (fix_ctas < 1 ? 1 : fix_ctas) : sms),
                                      kFixThreads, fix_smem, st>>>(a);
   count_launch();
