@@ -89,14 +89,17 @@ WORKLOADS = {
 # Captured on the Llama-shaped cache at context 8192 (1 layer, 524,288 vectors
 # per call); at that size part of a call's output is still in L2 when the
 # kernel ends, so the write bytes are a lower bound. The quantise entries sum
-# the main kernel and its fixup (the call the roofline times).
+# the main kernel and its fixup (the call the roofline times). The quantise
+# entries' sha covers a later change of the fixup's grid size only (host code;
+# the kernels' device code is the captured one, and the fixup reads the flag
+# words and the flagged rows once whatever its grid).
 TRAFFIC = {
     "decode_fused3_d128": {"bytes_per_unit": (65_936_640 + 58_624) / 524_288, "sha": "d958b2d61582ac83",
                            "sources": ["tq_decode_tc.cu", "tq_decode_tc.h", "tq_sm100.cuh"]},
     "quantize_tc_key3_d128": {"bytes_per_unit": (134_523_136 + 17_896_448 + 2_691_072) / 524_288,
-                              "sha": "466b735e2112a69a", "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
+                              "sha": "6813150f16aa91eb", "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
     "quantize_tc_value3_d128": {"bytes_per_unit": (134_339_072 + 9_486_336 + 2_416_640) / 524_288,
-                                "sha": "466b735e2112a69a",
+                                "sha": "6813150f16aa91eb",
                                 "sources": ["tq_quantize_tc.cu", "tq_tc.h", "tq_sm100.cuh"]},
 }
 
